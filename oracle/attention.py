@@ -1,0 +1,223 @@
+"""Plain, slow, fp64 CPU oracle for exact scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the library imports this module; only the
+test-suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
+call it.  It shares no code with the CUDA path.
+
+Sources (the three web pages on exact tiled attention):
+
+* "Atención Flash: Revolucionando la Eficiencia de los Modelos de Transformador"
+  (unite.ai), section "Atención Flash" / standard attention listing: the
+  definition softmax(Q K^T / sqrt(d_k)) V, with the score tensor of shape
+  (batch, seq, seq) materialised.  ``attention_fwd_ref`` is that definition,
+  written out in fp64, one (batch, head) at a time.
+* same page, section "La Matemática detrás de la Atención Flash", formula 1
+  (softmax decomposition with the row maximum m) and formula 2 (the merge of two
+  blocks with m = max(m_x, m_y)).  ``safe_softmax`` and ``softmax_merge``.
+* same page, section "Detalles de Implementación" (the simplified tiled loop):
+  running statistics M (max) and L (sum), query blocks outside, key/value blocks
+  inside.  ``online_softmax_attention`` restates that loop with the output update
+  corrected (the printed update drops the factor L of the old sum; here the old
+  output is multiplied by L * exp(M - M_new) before the division by L_new).
+* "FlashAttention algorithm part 3" (nisoo.com), sections "Softmax Sicura" and
+  "SafeSoftmax con Calcolo Normalizzatore Online": subtract the maximum before
+  exponentiating; keep a running normaliser corrected when the maximum moves.
+
+Not on the pages, taken from the method's statement of the task: the causal mask
+(key j visible to query i iff j <= i, square and top-left aligned), the per-row
+log-sum-exp output (natural log, of the scaled scores) and the backward pass
+(the closed-form softmax Jacobian).
+
+All arrays are numpy float64 with layout [B, H, N, d] (LSE: [B, H, N]).
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "safe_softmax",
+    "softmax_merge",
+    "scores",
+    "attention_fwd_ref",
+    "attention_bwd_ref",
+    "attention_rows_ref",
+    "online_softmax_attention",
+]
+
+
+def _as64(x):
+    return np.asarray(x, dtype=np.float64)
+
+
+def safe_softmax(x, axis=-1):
+    """softmax(x) = exp(x - m) / sum(exp(x - m)), m = max(x).
+
+    Softmax decomposition, formula 1 of the unite.ai page ("La Matemática detrás
+    de la Atención Flash"); the nisoo.com page ("Softmax Sicura") gives the same
+    rule in words.  Entries equal to -inf get probability 0.
+    """
+    x = _as64(x)
+    m = np.max(x, axis=axis, keepdims=True)
+    e = np.exp(x - m)
+    return e / np.sum(e, axis=axis, keepdims=True)
+
+
+def softmax_merge(fx, mx, lx, fy, my, ly):
+    """Merge the partial softmax statistics of two blocks x and y.
+
+    Formula 2 of the unite.ai page ("Fusión de Softmax"), whose printed form is
+    garbled.  Reading used here: for a block z keep f(z) = exp(z - m_z) and
+    l(z) = sum f(z).  With m = max(m_x, m_y):
+        f(x u y) = [exp(m_x - m) f(x), exp(m_y - m) f(y)]
+        l(x u y) = exp(m_x - m) l(x) + exp(m_y - m) l(y)
+        softmax(x u y) = f(x u y) / l(x u y)
+    Returns (softmax(x u y), m, l).
+    """
+    m = max(mx, my)
+    ax = math.exp(mx - m)
+    ay = math.exp(my - m)
+    f = np.concatenate([ax * _as64(fx), ay * _as64(fy)])
+    l = ax * lx + ay * ly
+    return f / l, m, l
+
+
+def scores(q, k, scale, causal):
+    """S = scale * Q K^T per (batch, head), with the causal mask applied.
+
+    The score tensor of the standard-attention listing (unite.ai page), here
+    one [N, N] matrix per (b, h).  Masked entries are -inf.
+    """
+    q = _as64(q)
+    k = _as64(k)
+    s = scale * np.einsum("bhid,bhjd->bhij", q, k)
+    if causal:
+        n = q.shape[2]
+        above = np.triu(np.ones((n, n), dtype=bool), k=1)
+        s = np.where(above, -np.inf, s)
+    return s
+
+
+def attention_fwd_ref(q, k, v, scale, causal):
+    """O = softmax(scale * Q K^T) V and LSE = log sum_j exp(scale * q_i . k_j).
+
+    The standard-attention definition of the unite.ai page, evaluated in fp64
+    with the full score matrix materialised.  LSE_i = m_i + ln sum_j
+    exp(S_ij - m_i) with m_i the row maximum (safe softmax).
+    """
+    v = _as64(v)
+    s = scores(q, k, scale, causal)
+    m = np.max(s, axis=-1, keepdims=True)
+    lse = m + np.log(np.sum(np.exp(s - m), axis=-1, keepdims=True))
+    p = np.exp(s - lse)
+    o = np.einsum("bhij,bhjd->bhid", p, v)
+    return o, lse[..., 0]
+
+
+def attention_bwd_ref(q, k, v, do, scale, causal):
+    """Gradients of L = sum(O * dO) with respect to Q, K and V.
+
+    Not on the pages; the closed form of the softmax Jacobian:
+        P   = softmax(S)            (row-wise)
+        dV  = P^T dO
+        dP  = dO V^T
+        dS  = P * (dP - rowsum(P * dP))
+        dQ  = scale * dS K
+        dK  = scale * dS^T Q
+    """
+    q = _as64(q)
+    k = _as64(k)
+    v = _as64(v)
+    do = _as64(do)
+    s = scores(q, k, scale, causal)
+    m = np.max(s, axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    p = e / np.sum(e, axis=-1, keepdims=True)
+    dv = np.einsum("bhij,bhid->bhjd", p, do)
+    dp = np.einsum("bhid,bhjd->bhij", do, v)
+    ds = p * (dp - np.sum(p * dp, axis=-1, keepdims=True))
+    dq = scale * np.einsum("bhij,bhjd->bhid", ds, k)
+    dk = scale * np.einsum("bhij,bhid->bhjd", ds, q)
+    return dq, dk, dv
+
+
+def attention_rows_ref(q, k, v, rows, scale, causal):
+    """O and LSE for selected query rows only, without the full N x N matrix.
+
+    Same definition as ``attention_fwd_ref``, evaluated row by row: for each
+    (b, h) and each query index i in ``rows[h]`` (or ``rows`` when it is one
+    list for all heads) the score row S[i, :] (keys 0..i when causal) is formed,
+    then its safe softmax and the weighted sum of V.
+    Returns (o [B, H, R, d], lse [B, H, R]).
+    """
+    q = _as64(q)
+    k = _as64(k)
+    v = _as64(v)
+    b_, h_, n, d = q.shape
+    per_head = isinstance(rows, (list, tuple)) and len(rows) > 0 and np.ndim(rows[0]) == 1
+    r = len(rows[0]) if per_head else len(rows)
+    o = np.zeros((b_, h_, r, d))
+    lse = np.zeros((b_, h_, r))
+    for b in range(b_):
+        for h in range(h_):
+            sel = rows[h] if per_head else rows
+            for t, i in enumerate(sel):
+                i = int(i)
+                kk = k[b, h, : i + 1] if causal else k[b, h]
+                vv = v[b, h, : i + 1] if causal else v[b, h]
+                srow = scale * (kk @ q[b, h, i])
+                m = np.max(srow)
+                e = np.exp(srow - m)
+                l = np.sum(e)
+                o[b, h, t] = (e / l) @ vv
+                lse[b, h, t] = m + math.log(l)
+    return o, lse
+
+
+def online_softmax_attention(q, k, v, scale, causal, block_q=128, block_k=128):
+    """The tiled loop of the unite.ai page ("Detalles de Implementación"), corrected.
+
+    Query blocks outside, key/value blocks inside; running maximum M and running
+    sum L per query row (initialised to -inf and 0), updated block by block with
+    exp(M - M_new) (formula 2 of the same page; the online normaliser of the
+    nisoo.com page).  The printed output update omits the factor L of the old
+    sum; here O_new = (L * exp(M - M_new) * O + exp(S - M_new) V) / L_new.
+    Returns (o, lse) so it can be compared with ``attention_fwd_ref``.
+    """
+    q = _as64(q)
+    k = _as64(k)
+    v = _as64(v)
+    b_, h_, n, d = q.shape
+    o = np.zeros_like(q)
+    lse = np.zeros((b_, h_, n))
+    for b in range(b_):
+        for h in range(h_):
+            for i0 in range(0, n, block_q):
+                i1 = min(n, i0 + block_q)
+                qb = q[b, h, i0:i1]
+                ob = np.zeros((i1 - i0, d))
+                mrow = np.full((i1 - i0, 1), -np.inf)
+                lrow = np.zeros((i1 - i0, 1))
+                for j0 in range(0, n, block_k):
+                    j1 = min(n, j0 + block_k)
+                    sb = scale * (qb @ k[b, h, j0:j1].T)
+                    if causal:
+                        qi = np.arange(i0, i1)[:, None]
+                        kj = np.arange(j0, j1)[None, :]
+                        sb = np.where(kj > qi, -np.inf, sb)
+                    m_new = np.maximum(mrow, np.max(sb, axis=-1, keepdims=True))
+                    # a row whose max is still -inf has seen no visible key yet
+                    safe_m = np.where(np.isneginf(m_new), 0.0, m_new)
+                    e = np.exp(sb - safe_m)
+                    corr = np.exp(mrow - safe_m)
+                    l_new = corr * lrow + np.sum(e, axis=-1, keepdims=True)
+                    with np.errstate(invalid="ignore", divide="ignore"):
+                        ob = np.where(
+                            l_new > 0, (lrow * corr * ob + e @ v[b, h, j0:j1]) / l_new, 0.0
+                        )
+                    mrow, lrow = m_new, l_new
+                o[b, h, i0:i1] = ob
+                lse[b, h, i0:i1] = (mrow + np.log(lrow))[:, 0]
+    return o, lse
