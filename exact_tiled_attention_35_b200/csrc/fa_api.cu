@@ -1,0 +1,188 @@
+// C ABI of libfa.so (declared in include/fa.h): argument checks, tensor-map
+// construction and kernel dispatch.  Every entry point validates on the host
+// before touching the device, so a bad argument never reaches a kernel.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "fa_device.cuh"
+#include "fa_kernels.h"
+
+namespace fa {
+
+__device__ unsigned int g_device_status = 0;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Checks shared by every entry point; no CUDA call is made.
+fa_status check_shape(int B, int H, int N, int d, float scale) {
+  if (B <= 0 || H <= 0 || N <= 0) return FA_ERR_INVALID_ARG;
+  if ((long long)B * H > 65535LL * 128) return FA_ERR_INVALID_ARG;
+  if ((long long)B * H * N * d >= (1LL << 40)) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+fa_status check_ptrs(std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs)
+    if (p == nullptr) return FA_ERR_INVALID_ARG;
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return FA_ERR_MISALIGNED;
+  return FA_OK;
+}
+
+size_t ws_bytes_for(int B, int H, int N) {
+  const size_t rows = (size_t)B * H * N;
+  return ((rows * sizeof(float)) + 255) / 256 * 256;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode;
+}
+
+// 3-D bf16 view {d, N, B*H} of a [B,H,N,d] tensor, box {64, 128, 1}, 128-byte
+// swizzle; rows past N read as zero.
+bool make_map(CUtensorMap* map, const void* base, int d, int N, int BH) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The tcgen05 kernels need an sm_100 device (compute capability 10.0).
+fa_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (major != 10 || minor != 0) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+fa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+fa_status fa_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                     int N, int d, float scale, int causal, void* stream) {
+  fa_status s = check_shape(B, H, N, d, scale);
+  if (s != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, o, lse})) != FA_OK) return s;
+  if ((s = check_device()) != FA_OK) return s;
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, d, N, BH) || !make_map(&mk, k, d, N, BH) || !make_map(&mv, v, d, N, BH))
+    return FA_ERR_CUDA;
+  return from_cuda(sm100_forward(mq, mk, mv, o, lse, BH, N, d, scale, causal ? 1 : 0,
+                                 static_cast<cudaStream_t>(stream)));
+}
+
+fa_status fa_forward_fp32(const float* q, const float* k, const float* v, float* o, float* lse, int B,
+                          int H, int N, int d, float scale, int causal, void* stream) {
+  fa_status s = check_shape(B, H, N, d, scale);
+  if (s != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, o, lse})) != FA_OK) return s;
+  return from_cuda(simt_forward(false, q, k, v, o, lse, B * H, N, d, scale, causal ? 1 : 0,
+                                static_cast<cudaStream_t>(stream)));
+}
+
+size_t fa_backward_workspace_size(int B, int H, int N, int d) {
+  if (check_shape(B, H, N, d, 1.0f) != FA_OK) return 0;
+  return ws_bytes_for(B, H, N);
+}
+
+fa_status fa_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                      const float* lse, void* dq, void* dk, void* dv, void* workspace,
+                      size_t ws_bytes, int B, int H, int N, int d, float scale, int causal,
+                      void* stream) {
+  fa_status s = check_shape(B, H, N, d, scale);
+  if (s != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv})) != FA_OK) return s;
+  if (workspace == nullptr || ws_bytes < ws_bytes_for(B, H, N)) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  if ((s = check_device()) != FA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* dsum = static_cast<float*>(workspace);
+  const int BH = B * H;
+  cudaError_t e = bwd_preprocess(true, o, dout, dsum, (long long)BH * N, d, st);
+  if (e != cudaSuccess) return FA_ERR_CUDA;
+  return from_cuda(simt_backward(true, q, k, v, dout, lse, dsum, dq, dk, dv, BH, N, d, scale,
+                                 causal ? 1 : 0, st));
+}
+
+fa_status fa_backward_fp32(const float* q, const float* k, const float* v, const float* o,
+                           const float* dout, const float* lse, float* dq, float* dk, float* dv,
+                           void* workspace, size_t ws_bytes, int B, int H, int N, int d, float scale,
+                           int causal, void* stream) {
+  fa_status s = check_shape(B, H, N, d, scale);
+  if (s != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv})) != FA_OK) return s;
+  if (workspace == nullptr || ws_bytes < ws_bytes_for(B, H, N)) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* dsum = static_cast<float*>(workspace);
+  const int BH = B * H;
+  cudaError_t e = bwd_preprocess(false, o, dout, dsum, (long long)BH * N, d, st);
+  if (e != cudaSuccess) return FA_ERR_CUDA;
+  return from_cuda(simt_backward(false, q, k, v, dout, lse, dsum, dq, dk, dv, BH, N, d, scale,
+                                 causal ? 1 : 0, st));
+}
+
+fa_status fa_check_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, g_device_status, sizeof(word)) != cudaSuccess) return FA_ERR_CUDA;
+  if (word != 0 && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return word ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
+}
+
+const char* fa_status_string(fa_status status) {
+  switch (status) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported head dimension or device";
+    case FA_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case FA_ERR_WORKSPACE: return "workspace missing or too small";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_DEVICE_TIMEOUT: return "a kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,385 @@
+// Forward pass on sm_100a: TMA-fed shared-memory ring, tcgen05 MMAs with fp32
+// accumulators in tensor memory, warp-specialised roles.
+//
+// What it computes is the standard attention of the page "Atención Flash:
+// Revolucionando la Eficiencia de los Modelos de Transformador" (unite.ai),
+// evaluated tile by tile as in its section "Detalles de Implementación": query
+// tiles outside (one CTA owns two 128-row query tiles), key/value tiles inside,
+// per-row running maximum m and running sum l, and the output rescaled by
+// exp(m_old - m_new) when m moves (formula 2, "Fusión de Softmax", of the same
+// page; the online normaliser of "FlashAttention algorithm part 3").  The output
+// stays unnormalised until the last tile and is divided by l once.  Tile size
+// 128 follows the block size the nisoo.com page reports as typical.
+//
+// CTA layout (320 threads):
+//   warps 0-3  softmax + epilogue for query tile 0 (tensor-memory lanes 0-127)
+//   warps 4-7  softmax + epilogue for query tile 1
+//   warp  8    TMA producer: Q tiles once, then K_j, V_j into a ring of slots
+//   warp  9    tensor-memory allocator and MMA issuer (one elected thread)
+// Tensor memory (512 columns): S_t at column 128*t (fp32 128x128, the bf16
+// probabilities P_t are written over its first 64 columns), O_t at 256 + D*t.
+// MMA order per key tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), so while one
+// softmax group works on its scores the tensor core runs the other's GEMMs.
+//
+// A row's maximum is only raised when it grows by more than 2^8 in the exp2
+// domain; P and l then use the same (stale) maximum, so O = O_acc / l and
+// LSE = m * scale + ln(l) stay exact up to fp32 rounding, and O is rescaled in
+// tensor memory only for those rows' warps.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "fa_device.cuh"
+#include "fa_kernels.h"
+
+namespace fa {
+namespace fwd {
+
+constexpr int BM = 128;           // query rows per tile
+constexpr int BN = 128;           // keys per tile
+constexpr int NQT = 2;            // query tiles per CTA
+constexpr int NTHREADS = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct Cfg {
+  static constexpr int TILE = BN * D * 2;          // bytes of one 128-row bf16 tile
+  static constexpr int CHUNK = BN * 128;           // bytes of one 64-column swizzle chunk
+  static constexpr int NSLOT = D == 128 ? 5 : 10;  // K/V ring slots
+  static constexpr int SMEM_Q = NQT * TILE;
+  static constexpr int SMEM_RING = NSLOT * TILE;
+  static constexpr int OFF_BAR = SMEM_Q + SMEM_RING;
+  static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;  // barriers + alignment slack
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, 0, 0);
+  static constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, 0, 1);
+};
+
+struct Params {
+  __nv_bfloat16* o;
+  float* lse;
+  int BH;
+  int N;
+  int npairs;  // ceil(N / 256)
+  float scale;
+  float scale_log2;
+  int causal;
+};
+
+struct Bars {
+  uint64_t q_full[NQT];
+  uint64_t s_full[NQT];
+  uint64_t p_full[NQT];
+  uint64_t o_full;
+  uint64_t drain;
+  uint64_t kv_full[16];
+  uint64_t kv_empty[16];
+  uint32_t tmem_base;
+};
+
+// number of key tiles query tile starting at row q0 needs (0 if the tile is empty)
+__device__ __forceinline__ int tiles_for(int q0, int N, int causal) {
+  if (q0 >= N) return 0;
+  const int nkv = (N + BN - 1) / BN;
+  if (!causal) return nkv;
+  return min(nkv, q0 / BN + 1);
+}
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+               const __grid_constant__ CUtensorMap mv, const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sQ = smem;
+  uint8_t* sRing = smem + C::SMEM_Q;
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  // heavy tiles first under the causal mask: pair index runs backwards
+  const int blk = blockIdx.x;
+  const int bh = blk % p.BH;
+  const int pair = p.causal ? (p.npairs - 1 - blk / p.BH) : (blk / p.BH);
+  const int qbase = pair * (NQT * BM);
+  int ntile[NQT];
+#pragma unroll
+  for (int t = 0; t < NQT; ++t) ntile[t] = tiles_for(qbase + t * BM, p.N, p.causal);
+  const int nmax = max(ntile[0], ntile[1]);
+
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int t = 0; t < NQT; ++t) {
+      mbar_init(&bars->q_full[t], 1);
+      mbar_init(&bars->s_full[t], 1);
+      mbar_init(&bars->p_full[t], 128);
+    }
+    mbar_init(&bars->o_full, 1);
+    mbar_init(&bars->drain, 1);
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    tma_prefetch_desc(&mq);
+    tma_prefetch_desc(&mk);
+    tma_prefetch_desc(&mv);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      bool ok = true;
+      for (int t = 0; t < NQT; ++t) {
+        if (ntile[t] == 0) continue;
+        mbar_arrive_expect_tx(&bars->q_full[t], C::TILE);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &mq, &bars->q_full[t], c * 64,
+                      qbase + t * BM, bh);
+      }
+      // ring sequence: K_0, V_0, K_1, V_1, ...
+      int issued = 0;
+      for (int seq = 0; seq < 2 * nmax && ok; ++seq) {
+        const int slot = seq % C::NSLOT, round = seq / C::NSLOT;
+        if (round > 0) ok = mbar_wait(&bars->kv_empty[slot], (round - 1) & 1, 1);
+        if (!ok) break;
+        const int j = seq >> 1;
+        const CUtensorMap* m = (seq & 1) ? &mv : &mk;
+        uint8_t* dst = sRing + slot * C::TILE;
+        mbar_arrive_expect_tx(&bars->kv_full[slot], C::TILE);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(dst + c * C::CHUNK, m, &bars->kv_full[slot], c * 64, j * BN, bh);
+        issued = seq + 1;
+      }
+      // make sure no copy into this CTA's shared memory is still in flight at exit
+      for (int s = 0; s < C::NSLOT && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / C::NSLOT) * C::NSLOT;
+        mbar_wait(&bars->kv_full[s], (last / C::NSLOT) & 1, 2);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      bool ok = true;
+      const uint32_t sq = smem_u32(sQ), sr = smem_u32(sRing);
+      auto slot_of = [&](int seq) { return seq % C::NSLOT; };
+      auto phase_of = [&](int seq) { return (uint32_t)((seq / C::NSLOT) & 1); };
+      // S_t = Q_t K_j^T : A = Q_t (K-major), B = K_j (K-major), K = D in steps of 16
+      auto issue_s = [&](int t, int j) {
+        const uint32_t a0 = sq + t * C::TILE, b0 = sr + slot_of(2 * j) * C::TILE;
+        const uint32_t d_tmem = tmem + t * BN;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+          mma_ss(d_tmem, sdesc_sw128(a0 + koff, 16, 1024), sdesc_sw128(b0 + koff, 16, 1024),
+                 C::IDESC_QK, kk > 0);
+        }
+      };
+      // O_t += P_t V_j : A = P_t (tensor memory), B = V_j (MN-major), K = 128 keys
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t b0 = sr + slot_of(2 * j + 1) * C::TILE;
+        const uint32_t d_tmem = tmem + 2 * BN + t * D;
+        const uint32_t a_tmem = tmem + t * BN;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b0 + kk * 16 * 128, C::CHUNK, 1024),
+                 C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      for (int t = 0; t < NQT && ok; ++t)
+        if (ntile[t] > 0) ok = mbar_wait(&bars->q_full[t], 0, 3);
+      if (ok && nmax > 0) ok = mbar_wait(&bars->kv_full[slot_of(0)], phase_of(0), 4);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < NQT; ++t)
+          if (ntile[t] > 0) {
+            issue_s(t, 0);
+            mma_commit(&bars->s_full[t]);
+          }
+        if (nmax > 0) mma_commit(&bars->kv_empty[slot_of(0)]);
+      }
+      for (int j = 0; j < nmax && ok; ++j) {
+        ok = mbar_wait(&bars->kv_full[slot_of(2 * j + 1)], phase_of(2 * j + 1), 5);
+        bool k_next_ready = false;
+        for (int t = 0; t < NQT && ok; ++t) {
+          if (j >= ntile[t]) continue;
+          ok = mbar_wait(&bars->p_full[t], j & 1, 6);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(t, j);
+          if (j + 1 < ntile[t]) {
+            if (!k_next_ready) {
+              ok = mbar_wait(&bars->kv_full[slot_of(2 * j + 2)], phase_of(2 * j + 2), 7);
+              if (!ok) break;
+              tc_fence_after();
+              k_next_ready = true;
+            }
+            issue_s(t, j + 1);
+            mma_commit(&bars->s_full[t]);
+          }
+        }
+        if (!ok) break;
+        mma_commit(&bars->kv_empty[slot_of(2 * j + 1)]);
+        if (k_next_ready) mma_commit(&bars->kv_empty[slot_of(2 * j + 2)]);
+      }
+      if (ok) mma_commit(&bars->o_full);
+      // wait for every MMA this thread issued before tensor memory is released
+      mma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, 8);
+    }
+  } else {
+    // softmax / epilogue groups
+    const int t = warp / 4;
+    const int row = (warp % 4) * 32 + lane;
+    const int q_row = qbase + t * BM + row;
+    const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * BN;
+    const uint32_t tO = tmem + lane_off + 2 * BN + t * D;
+    const float c = p.scale_log2;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    const int n = ntile[t];
+    for (int j = 0; j < n && ok; ++j) {
+      ok = mbar_wait(&bars->s_full[t], j & 1, 16 + t);
+      if (!ok) break;
+      tc_fence_after();
+      float s[BN];
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tS + cc * 32, r);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[cc * 32 + i] = __uint_as_float(r[i]);
+      }
+      tmem_wait_ld();
+      const int k0 = j * BN;
+      const bool need_mask = (p.causal && j == n - 1) || (k0 + BN > p.N);
+      if (need_mask) {
+        const int lim = p.causal ? min(q_row + 1, p.N) : p.N;  // keys < lim are visible
+#pragma unroll
+        for (int i = 0; i < BN; ++i)
+          if (k0 + i >= lim) s[i] = -INFINITY;
+      }
+      float mx4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+      for (int i = 4; i < BN; ++i) mx4[i % 4] = fmaxf(mx4[i % 4], s[i]);
+      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      const float m_new = fmaxf(m_used, mx);
+      const bool need = (m_new - m_used) * c > kRescaleThreshold;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2((m_used - m_new) * c);
+        m_used = m_new;
+      }
+      // a row that has seen no visible key keeps m = -inf; pivot on 0 then
+      const float mc = m_used == -INFINITY ? 0.f : m_used * c;
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[BN / 2];
+#pragma unroll
+      for (int i = 0; i < BN / 2; ++i) {
+        const float p0 = ex2(fmaf(s[2 * i], c, -mc));
+        const float p1 = ex2(fmaf(s[2 * i + 1], c, -mc));
+        sum4[i % 4] += p0 + p1;
+        pk[i] = pack_bf16x2(p0, p1);
+      }
+      l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(tO + cc * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(tO + cc * 32, r);
+        }
+      }
+#pragma unroll
+      for (int cc = 0; cc < BN / 64; ++cc) {
+        uint32_t r[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) r[i] = pk[cc * 32 + i];
+        tmem_st32(tS + cc * 32, r);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[t]);
+    }
+    if (ok && n > 0) ok = mbar_wait(&bars->o_full, 0, 20 + t);
+    if (ok && n > 0) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (size_t)(q_row < p.N ? q_row : 0)) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t r[32];
+        tmem_ld32(tO + cc * 32, r);
+        tmem_wait_ld();
+        if (q_row < p.N) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+      if (q_row < p.N)
+        p.lse[(size_t)bh * p.N + q_row] = l > 0.f ? m_used * p.scale + logf(l) : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fwd
+
+cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                          void* o, float* lse, int BH, int N, int d, float scale, int causal,
+                          cudaStream_t st) {
+  fwd::Params p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.BH = BH;
+  p.N = N;
+  p.npairs = (N + 2 * fwd::BM - 1) / (2 * fwd::BM);
+  p.scale = scale;
+  p.scale_log2 = scale * fwd::kLog2e;
+  p.causal = causal;
+  const dim3 grid((unsigned)(p.npairs * BH));
+  cudaError_t e;
+  if (d == 128) {
+    const int smem = fwd::Cfg<128>::SMEM_BYTES;
+    e = cudaFuncSetAttribute(fwd::fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    fwd::fwd_kernel<128><<<grid, fwd::NTHREADS, smem, st>>>(mq, mk, mv, p);
+  } else {
+    const int smem = fwd::Cfg<64>::SMEM_BYTES;
+    e = cudaFuncSetAttribute(fwd::fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    fwd::fwd_kernel<64><<<grid, fwd::NTHREADS, smem, st>>>(mq, mk, mv, p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace fa

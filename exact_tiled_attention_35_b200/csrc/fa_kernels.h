@@ -1,0 +1,24 @@
+// Internal launch entry points of the kernels (host side).  Not part of the ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+// CUDA-core kernels (fa_simt.cu)
+cudaError_t simt_forward(bool bf16, const void* q, const void* k, const void* v, void* o, float* lse,
+                         int BH, int N, int d, float scale, int causal, cudaStream_t st);
+cudaError_t bwd_preprocess(bool bf16, const void* o, const void* dout, float* dsum, long long rows,
+                           int d, cudaStream_t st);
+cudaError_t simt_backward(bool bf16, const void* q, const void* k, const void* v, const void* dout,
+                          const float* lse, const float* dsum, void* dq, void* dk, void* dv, int BH,
+                          int N, int d, float scale, int causal, cudaStream_t st);
+
+// tcgen05 forward (fa_fwd_sm100.cu).  Tensor maps: 3-D bf16 views
+// {d, N, B*H} of Q, K, V with a {64, 128, 1} box and 128-byte swizzle.
+cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                          void* o, float* lse, int BH, int N, int d, float scale, int causal,
+                          cudaStream_t st);
+
+}  // namespace fa

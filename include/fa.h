@@ -1,0 +1,104 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact tiled (FlashAttention-style) attention for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  For every batch b and head h, with S = scale * Q K^T
+ * (Q, K, V of shape N x d), the exact attention
+ *     O   = softmax(S) V
+ *     LSE = log(sum_j exp(S_ij))          (natural log, per query row i)
+ * as defined by the standard-attention listing of the page "Atención Flash:
+ * Revolucionando la Eficiencia de los Modelos de Transformador" (unite.ai),
+ * section "Atención Flash", evaluated block by block with a running row maximum
+ * m and running sum l (same page, "La Matemática detrás de la Atención Flash",
+ * formulas 1-2, and "Detalles de Implementación"; page "FlashAttention
+ * algorithm part 3" (nisoo.com), "SafeSoftmax con Calcolo Normalizzatore
+ * Online"), so the N x N score matrix never reaches device memory.  With
+ * causal != 0, key j is visible to query i only when j <= i (square, top-left
+ * aligned).  The backward pass recomputes the score blocks from Q, K and the
+ * saved LSE (the "recomputation" idea of both pages) and returns dQ, dK, dV of
+ * L = sum(O * dO).
+ *
+ * Layout.  Q, K, V, O, dO, dQ, dK, dV: [B, H, N, d] contiguous, row-major
+ * (d fastest).  LSE: [B, H, N] float32, contiguous.
+ *
+ * Ownership.  Every pointer is caller-owned DEVICE memory on the current CUDA
+ * device.  The library allocates nothing; the backward pass's scratch comes
+ * from the caller (fa_backward_workspace_size).
+ *
+ * Asynchrony.  Work is enqueued on `stream` (a cudaStream_t; 0 = legacy
+ * default stream) and the call returns at once.  The returned status covers
+ * argument checks and launch errors.  Kernels bound every wait they make; a
+ * wait that runs out records FA_ERR_DEVICE_TIMEOUT in a device-side status
+ * word instead of hanging, which fa_check_device_status reports.
+ *
+ * Limits.  d in {64, 128}; N >= 1 (any N: ragged tails are masked);
+ * 1 <= B*H <= 65535*128; pointers 16-byte aligned; scale finite and > 0.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, bad scale */
+  FA_ERR_UNSUPPORTED = 2,    /* head dim / device not supported */
+  FA_ERR_MISALIGNED = 3,     /* a pointer is not 16-byte aligned */
+  FA_ERR_WORKSPACE = 4,      /* workspace missing or smaller than required */
+  FA_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
+  FA_ERR_DEVICE_TIMEOUT = 6  /* a kernel's bounded wait ran out */
+} fa_status;
+
+/* Forward pass, bf16 storage, fp32 accumulation and statistics.
+ * q, k, v: const bf16 [B,H,N,d]; o: bf16 [B,H,N,d] (written); lse: fp32
+ * [B,H,N] (written).  scale multiplies Q K^T (1/sqrt(d) for the pages'
+ * scaled dot product).  Runs the tcgen05/TMEM/TMA kernel on sm_100a. */
+fa_status fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/* Forward pass with fp32 storage (q, k, v, o are float [B,H,N,d]); fp32
+ * arithmetic on CUDA cores.  Same definition, same LSE convention. */
+fa_status fa_forward_fp32(const float* q, const float* k, const float* v, float* o, float* lse,
+                          int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/* Bytes of device scratch fa_backward needs for this shape (0 on bad sizes).
+ * It holds D_i = sum_c dO[i,c] * O[i,c] (fp32, [B,H,N]). */
+size_t fa_backward_workspace_size(int B, int H, int N, int d);
+
+/* Backward pass, bf16 storage, fp32 accumulation.
+ * q, k, v, o, dout: const bf16 [B,H,N,d] (o and lse as written by fa_forward
+ * for the same q, k, v, scale, causal); lse: const fp32 [B,H,N];
+ * dq, dk, dv: bf16 [B,H,N,d] (written);
+ * workspace: device scratch of ws_bytes >= fa_backward_workspace_size(...),
+ * 16-byte aligned, contents ignored on entry and undefined on return.
+ * Computes dV = P^T dO, dP = dO V^T, dS = P * (dP - rowsum(dO * O)),
+ * dQ = scale * dS K, dK = scale * dS^T Q with P recomputed from Q, K and LSE. */
+fa_status fa_backward(const void* q, const void* k, const void* v, const void* o,
+                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                      void* workspace, size_t ws_bytes, int B, int H, int N, int d,
+                      float scale, int causal, void* stream);
+
+/* Backward pass with fp32 storage (all tensors float); CUDA-core arithmetic.
+ * Workspace as for fa_backward. */
+fa_status fa_backward_fp32(const float* q, const float* k, const float* v, const float* o,
+                           const float* dout, const float* lse, float* dq, float* dk, float* dv,
+                           void* workspace, size_t ws_bytes, int B, int H, int N, int d,
+                           float scale, int causal, void* stream);
+
+/* Synchronises `stream`, then reads and clears the current device's status
+ * word.  FA_ERR_DEVICE_TIMEOUT if a kernel gave up a wait since the last call;
+ * FA_ERR_CUDA if synchronisation failed; FA_OK otherwise. */
+fa_status fa_check_device_status(void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* fa_status_string(fa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

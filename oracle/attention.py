@@ -92,7 +92,7 @@ def scores(q, k, scale, causal):
     """
     q = _as64(q)
     k = _as64(k)
-    s = scale * np.einsum("bhid,bhjd->bhij", q, k)
+    s = scale * np.matmul(q, np.swapaxes(k, -1, -2))
     if causal:
         n = q.shape[2]
         above = np.triu(np.ones((n, n), dtype=bool), k=1)
@@ -112,7 +112,7 @@ def attention_fwd_ref(q, k, v, scale, causal):
     m = np.max(s, axis=-1, keepdims=True)
     lse = m + np.log(np.sum(np.exp(s - m), axis=-1, keepdims=True))
     p = np.exp(s - lse)
-    o = np.einsum("bhij,bhjd->bhid", p, v)
+    o = np.matmul(p, v)
     return o, lse[..., 0]
 
 
@@ -135,11 +135,11 @@ def attention_bwd_ref(q, k, v, do, scale, causal):
     m = np.max(s, axis=-1, keepdims=True)
     e = np.exp(s - m)
     p = e / np.sum(e, axis=-1, keepdims=True)
-    dv = np.einsum("bhij,bhid->bhjd", p, do)
-    dp = np.einsum("bhid,bhjd->bhij", do, v)
+    dv = np.matmul(np.swapaxes(p, -1, -2), do)
+    dp = np.matmul(do, np.swapaxes(v, -1, -2))
     ds = p * (dp - np.sum(p * dp, axis=-1, keepdims=True))
-    dq = scale * np.einsum("bhij,bhjd->bhid", ds, k)
-    dk = scale * np.einsum("bhij,bhid->bhjd", ds, q)
+    dq = scale * np.matmul(ds, k)
+    dk = scale * np.matmul(np.swapaxes(ds, -1, -2), q)
     return dq, dk, dv
 
 

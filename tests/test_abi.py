@@ -1,0 +1,93 @@
+"""Host-only checks of the C ABI: the library loads, exports every entry point
+declared in include/fa.h, and rejects bad arguments before touching a device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_tiled_attention_35_b200 as fa
+from exact_tiled_attention_35_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA, TIMEOUT = range(7)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return fa.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert set(declared_functions()) == set(fa.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in range(7):
+        assert fa.status_string(code)
+    assert fa.status_string(99) == "unknown status"
+
+
+P = ctypes.c_void_p
+GOOD = [P(0x10000), P(0x20000), P(0x30000), P(0x40000), P(0x50000)]
+
+
+def fwd(lib, ptrs, B=1, H=1, N=128, d=128, scale=0.125, causal=0, fn="fa_forward"):
+    return getattr(lib, fn)(*ptrs, B, H, N, d, scale, causal, None)
+
+
+@pytest.mark.parametrize("fn", ["fa_forward", "fa_forward_fp32"])
+def test_forward_rejects_bad_arguments(lib, fn):
+    for i in range(5):
+        ptrs = list(GOOD)
+        ptrs[i] = None
+        assert fwd(lib, ptrs, fn=fn) == INVALID
+    ptrs = list(GOOD)
+    ptrs[2] = P(0x30008)
+    assert fwd(lib, ptrs, fn=fn) == MISALIGNED
+    assert fwd(lib, GOOD, d=96, fn=fn) == UNSUPPORTED
+    assert fwd(lib, GOOD, d=256, fn=fn) == UNSUPPORTED
+    assert fwd(lib, GOOD, N=0, fn=fn) == INVALID
+    assert fwd(lib, GOOD, B=0, fn=fn) == INVALID
+    assert fwd(lib, GOOD, H=-1, fn=fn) == INVALID
+    assert fwd(lib, GOOD, scale=0.0, fn=fn) == INVALID
+    assert fwd(lib, GOOD, scale=float("nan"), fn=fn) == INVALID
+    assert fwd(lib, GOOD, scale=float("inf"), fn=fn) == INVALID
+
+
+def test_workspace_size(lib):
+    assert lib.fa_backward_workspace_size(2, 16, 2048, 128) == 2 * 16 * 2048 * 4
+    assert lib.fa_backward_workspace_size(1, 1, 3, 64) == 256
+    assert lib.fa_backward_workspace_size(1, 1, 3, 96) == 0
+    assert lib.fa_backward_workspace_size(0, 1, 3, 64) == 0
+
+
+@pytest.mark.parametrize("fn", ["fa_backward", "fa_backward_fp32"])
+def test_backward_rejects_bad_arguments(lib, fn):
+    ptrs = [P(0x10000 * (i + 1)) for i in range(9)]
+    ws = P(0x100000)
+    need = lib.fa_backward_workspace_size(1, 2, 300, 64)
+    f = getattr(lib, fn)
+    assert f(*ptrs, ws, need - 1, 1, 2, 300, 64, 0.125, 0, None) == WORKSPACE
+    assert f(*ptrs, None, need, 1, 2, 300, 64, 0.125, 0, None) == WORKSPACE
+    assert f(*ptrs, P(0x100004), need, 1, 2, 300, 64, 0.125, 0, None) == MISALIGNED
+    for i in range(9):
+        bad = list(ptrs)
+        bad[i] = None
+        assert f(*bad, ws, need, 1, 2, 300, 64, 0.125, 0, None) == INVALID
+    assert f(*ptrs, ws, need, 1, 2, 300, 80, 0.125, 0, None) == UNSUPPORTED
