@@ -41,9 +41,11 @@ fa_status check_ptrs(std::initializer_list<const void*> ptrs) {
   return FA_OK;
 }
 
-size_t ws_bytes_for(int B, int H, int N) {
-  const size_t rows = (size_t)B * H * N;
-  return ((rows * sizeof(float)) + 255) / 256 * 256;
+// Scratch of the bf16 (tcgen05) backward; the fp32 path uses a prefix of it.
+size_t ws_bytes_for(int B, int H, int N, int d) {
+  const size_t simt = ((size_t)B * H * N * sizeof(float) + 255) / 256 * 256;
+  const size_t tc = sm100_backward_workspace(B * H, N, d);
+  return simt > tc ? simt : tc;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
@@ -123,7 +125,7 @@ fa_status fa_forward_fp32(const float* q, const float* k, const float* v, float*
 
 size_t fa_backward_workspace_size(int B, int H, int N, int d) {
   if (check_shape(B, H, N, d, 1.0f) != FA_OK) return 0;
-  return ws_bytes_for(B, H, N);
+  return ws_bytes_for(B, H, N, d);
 }
 
 fa_status fa_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -133,16 +135,16 @@ fa_status fa_backward(const void* q, const void* k, const void* v, const void* o
   fa_status s = check_shape(B, H, N, d, scale);
   if (s != FA_OK) return s;
   if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv})) != FA_OK) return s;
-  if (workspace == nullptr || ws_bytes < ws_bytes_for(B, H, N)) return FA_ERR_WORKSPACE;
+  if (workspace == nullptr || ws_bytes < ws_bytes_for(B, H, N, d)) return FA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
   if ((s = check_device()) != FA_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  float* dsum = static_cast<float*>(workspace);
   const int BH = B * H;
-  cudaError_t e = bwd_preprocess(true, o, dout, dsum, (long long)BH * N, d, st);
-  if (e != cudaSuccess) return FA_ERR_CUDA;
-  return from_cuda(simt_backward(true, q, k, v, dout, lse, dsum, dq, dk, dv, BH, N, d, scale,
-                                 causal ? 1 : 0, st));
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, q, d, N, BH) || !make_map(&mk, k, d, N, BH) || !make_map(&mv, v, d, N, BH) ||
+      !make_map(&mdo, dout, d, N, BH))
+    return FA_ERR_CUDA;
+  return from_cuda(sm100_backward(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, workspace, BH, N, d,
+                                  scale, causal ? 1 : 0, static_cast<cudaStream_t>(stream)));
 }
 
 fa_status fa_backward_fp32(const float* q, const float* k, const float* v, const float* o,
@@ -152,7 +154,7 @@ fa_status fa_backward_fp32(const float* q, const float* k, const float* v, const
   fa_status s = check_shape(B, H, N, d, scale);
   if (s != FA_OK) return s;
   if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv})) != FA_OK) return s;
-  if (workspace == nullptr || ws_bytes < ws_bytes_for(B, H, N)) return FA_ERR_WORKSPACE;
+  if (workspace == nullptr || ws_bytes < ws_bytes_for(B, H, N, d)) return FA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* dsum = static_cast<float*>(workspace);

@@ -1,0 +1,530 @@
+// Backward pass on sm_100a.  The score tiles are recomputed from Q, K and the
+// saved LSE instead of being stored (the "recomputation" idea of the page
+// "Atención Flash: Revolucionando la Eficiencia de los Modelos de Transformador"
+// and of "FlashAttention algorithm part 3"); the gradient formulas are the
+// closed form of the softmax Jacobian:
+//   P = exp(S - LSE),  dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),
+//   D_i = sum_c dO[i,c] O[i,c],  dQ = scale * dS K,  dK = scale * dS^T Q.
+//
+// Three kernels:
+//   preprocess  D, LSE * log2(e) (padded to whole 128-row tiles: padding rows get
+//               LSE = +inf so their probabilities vanish) and a zeroed fp32 dQ
+//               accumulator;
+//   main        one CTA per 128-key tile; for every 128-row query tile it
+//               recomputes S^T = K Q^T and dP^T = V dO^T in tensor memory,
+//               forms P^T (to tensor memory) and dS (to shared memory), then
+//               accumulates dV += P^T dO and dK += dS^T Q in tensor memory and
+//               computes the partial dQ = dS K, which a reduce group adds into
+//               the fp32 accumulator with vector atomics;
+//   convert     dQ = scale * accumulator, rounded to bf16.
+//
+// Main-kernel CTA layout (320 threads):
+//   warps 0-3  P / dS computation (thread = key row = tensor-memory lane),
+//              then the dK / dV epilogue
+//   warps 4-7  dQ reduce: tensor memory -> registers -> red.global.add.v4.f32
+//   warp  8    TMA producer: K, V once; Q_i, dO_i, LSE_i, D_i per query tile
+//   warp  9    tensor-memory allocator and MMA issuer
+// Tensor memory: S^T / P^T at column 0, dP^T / dQ at 128, dV at 256, dK at 256+d.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "fa_device.cuh"
+#include "fa_kernels.h"
+
+namespace fa {
+namespace bwd {
+
+constexpr int BM = 128;  // query rows per tile
+constexpr int BN = 128;  // keys per tile
+constexpr int NTHREADS = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int NST = 2;  // Q / dO stages
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct Cfg {
+  static constexpr int TILE = BN * D * 2;  // bytes of one 128-row bf16 tile
+  static constexpr int CHUNK = BN * 128;   // one 64-column swizzle chunk of a tile
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = TILE;
+  static constexpr int OFF_STAGE = 2 * TILE;       // stage s: Q at +0, dO at +TILE
+  static constexpr int OFF_DS = OFF_STAGE + NST * 2 * TILE;
+  static constexpr int OFF_VEC = OFF_DS + BM * BN * 2;  // LSE2 / D vectors per stage
+  static constexpr int OFF_BAR = OFF_VEC + NST * 2 * BM * 4;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
+  static constexpr uint32_t IDESC_S = idesc_bf16(BN, BM, 0, 0);   // K-major x K-major
+  static constexpr uint32_t IDESC_DQ = idesc_bf16(BM, D, 1, 1);   // dS (MN) x K (MN)
+  static constexpr uint32_t IDESC_DKV = idesc_bf16(BN, D, 0, 1);  // P^T/dS^T (K) x dO/Q (MN)
+};
+
+struct Params {
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  float* dq_acc;       // [BH, N, d] fp32
+  const float* lse2;   // [BH, Npad]  LSE * log2(e), +inf on padding rows
+  const float* dsum;   // [BH, Npad]  D, 0 on padding rows
+  int BH;
+  int N;
+  int Npad;
+  int nkv;             // number of key tiles = Npad / 128
+  float scale;
+  float scale_log2;
+  int causal;
+};
+
+struct Bars {
+  uint64_t kv_full;
+  uint64_t qdo_full[NST];
+  uint64_t qdo_empty[NST];
+  uint64_t s_full;
+  uint64_t dp_full;
+  uint64_t ds_full;
+  uint64_t ds_free;
+  uint64_t dq_full;
+  uint64_t dq_empty;
+  uint64_t all_done;
+  uint64_t drain;
+  uint32_t tmem_base;
+};
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    main_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
+                const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  // The swizzled tiles need a 1024-byte aligned base and the layout uses the
+  // whole opt-in shared memory, so there is no slack to re-align: refuse to run
+  // on a misaligned base instead of computing garbage.
+  if (smem_u32(smem) & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(&g_device_status, 0u, 0x200u);
+    return;
+  }
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  uint8_t* sDS = smem + C::OFF_DS;
+  float* sVec = reinterpret_cast<float*>(smem + C::OFF_VEC);  // [NST][2][BM]
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  // heavy key tiles first under the causal mask (tile j sees query tiles j..)
+  const int blk = blockIdx.x;
+  const int bh = blk % p.BH;
+  const int j = blk / p.BH;
+  const int nq = p.nkv;
+  const int i0 = p.causal ? j : 0;
+  const int niter = nq - i0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kv_full, 1);
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&bars->qdo_full[s], 1);
+      mbar_init(&bars->qdo_empty[s], 1);
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->dp_full, 1);
+    mbar_init(&bars->ds_full, 128);
+    mbar_init(&bars->ds_free, 1);
+    mbar_init(&bars->dq_full, 1);
+    mbar_init(&bars->dq_empty, 128);
+    mbar_init(&bars->all_done, 1);
+    mbar_init(&bars->drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    tma_prefetch_desc(&mq);
+    tma_prefetch_desc(&mk);
+    tma_prefetch_desc(&mv);
+    tma_prefetch_desc(&mdo);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d(sK + c * C::CHUNK, &mk, &bars->kv_full, c * 64, j * BN, bh);
+        tma_load_3d(sV + c * C::CHUNK, &mv, &bars->kv_full, c * 64, j * BN, bh);
+      }
+      bool ok = true;
+      int issued = 0;
+      for (int it = 0; it < niter && ok; ++it) {
+        const int st = it % NST, round = it / NST;
+        if (round > 0) ok = mbar_wait(&bars->qdo_empty[st], (round - 1) & 1, 32);
+        if (!ok) break;
+        const int i = i0 + it;
+        uint8_t* sQ = smem + C::OFF_STAGE + st * 2 * C::TILE;
+        uint8_t* sdO = sQ + C::TILE;
+        float* vec = sVec + st * 2 * BM;
+        mbar_arrive_expect_tx(&bars->qdo_full[st], 2 * C::TILE + 2 * BM * 4);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(sQ + c * C::CHUNK, &mq, &bars->qdo_full[st], c * 64, i * BM, bh);
+          tma_load_3d(sdO + c * C::CHUNK, &mdo, &bars->qdo_full[st], c * 64, i * BM, bh);
+        }
+        const size_t voff = (size_t)bh * p.Npad + (size_t)i * BM;
+        bulk_load(vec, p.lse2 + voff, BM * 4, &bars->qdo_full[st]);
+        bulk_load(vec + BM, p.dsum + voff, BM * 4, &bars->qdo_full[st]);
+        issued = it + 1;
+      }
+      mbar_wait(&bars->kv_full, 0, 33);
+      for (int s = 0; s < NST && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / NST) * NST;
+        mbar_wait(&bars->qdo_full[s], (last / NST) & 1, 34);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      const uint32_t uK = smem_u32(sK), uV = smem_u32(sV), uDS = smem_u32(sDS);
+      bool ok = mbar_wait(&bars->kv_full, 0, 35);
+      for (int it = 0; it < niter && ok; ++it) {
+        const int st = it % NST;
+        const uint32_t uQ = smem_u32(smem + C::OFF_STAGE + st * 2 * C::TILE);
+        const uint32_t udO = uQ + C::TILE;
+        ok = mbar_wait(&bars->qdo_full[st], (it / NST) & 1, 36);
+        if (!ok) break;
+        tc_fence_after();
+        // S^T = K Q^T  (keys x queries), K = d
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+          mma_ss(tmem + C::T_S, sdesc_sw128(uK + ko, 16, 1024), sdesc_sw128(uQ + ko, 16, 1024),
+                 C::IDESC_S, kk > 0);
+        }
+        mma_commit(&bars->s_full);
+        if (it > 0) {
+          ok = mbar_wait(&bars->dq_empty, (it - 1) & 1, 37);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        // dP^T = V dO^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+          mma_ss(tmem + C::T_DP, sdesc_sw128(uV + ko, 16, 1024), sdesc_sw128(udO + ko, 16, 1024),
+                 C::IDESC_S, kk > 0);
+        }
+        mma_commit(&bars->dp_full);
+        ok = mbar_wait(&bars->ds_full, it & 1, 38);
+        if (!ok) break;
+        tc_fence_after();
+        // dQ_part = dS K  (queries x d), K = 128 keys; written over dP^T
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ss(tmem + C::T_DP, sdesc_sw128(uDS + kk * 2048, C::CHUNK, 1024),
+                 sdesc_sw128(uK + kk * 2048, C::CHUNK, 1024), C::IDESC_DQ, kk > 0);
+        mma_commit(&bars->dq_full);
+        // dV += P^T dO  (keys x d), K = 128 queries, P^T from tensor memory
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_ts(tmem + C::T_DV, tmem + C::T_S + kk * 8, sdesc_sw128(udO + kk * 2048, C::CHUNK, 1024),
+                 C::IDESC_DKV, (it > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q  (keys x d), K = 128 queries
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk) {
+          const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+          mma_ss(tmem + C::T_DK, sdesc_sw128(uDS + ko, 16, 1024),
+                 sdesc_sw128(uQ + kk * 2048, C::CHUNK, 1024), C::IDESC_DKV,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&bars->ds_free);
+        mma_commit(&bars->qdo_empty[st]);
+      }
+      if (ok) mma_commit(&bars->all_done);
+      mma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, 39);
+    }
+  } else if (warp < 4) {
+    // P^T and dS for key row r of this tile
+    const int r = warp * 32 + lane;
+    const int kr = j * BN + r;
+    const bool key_ok = kr < p.N;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::T_S;
+    const uint32_t tDP = tmem + lane_off + C::T_DP;
+    const float c = p.scale_log2;
+    const uint32_t ds_row = smem_u32(sDS) + r * 128;
+    bool ok = true;
+    for (int it = 0; it < niter && ok; ++it) {
+      const int i = i0 + it, st = it % NST;
+      const float* lse2 = sVec + st * 2 * BM;
+      const float* dsv = lse2 + BM;
+      ok = mbar_wait(&bars->qdo_full[st], (it / NST) & 1, 40);
+      if (ok) ok = mbar_wait(&bars->s_full, it & 1, 41);
+      if (!ok) break;
+      tc_fence_after();
+      float pr[BM];
+#pragma unroll
+      for (int cc = 0; cc < BM / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tS + cc * 32, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pr[cc * 32 + e] = __uint_as_float(v[e]);
+      }
+      tmem_wait_ld();
+      const bool diag = p.causal && i == j;
+#pragma unroll
+      for (int c4 = 0; c4 < BM / 4; ++c4) {
+        const float4 l4 = reinterpret_cast<const float4*>(lse2)[c4];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int col = c4 * 4 + e;
+          float pv = ex2(fmaf(pr[col], c, -lv[e]));
+          if (!key_ok || (diag && col < r)) pv = 0.f;
+          pr[col] = pv;
+        }
+      }
+#pragma unroll
+      for (int cc = 0; cc < BM / 64; ++cc) {
+        uint32_t v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = pack_bf16x2(pr[cc * 64 + 2 * e], pr[cc * 64 + 2 * e + 1]);
+        tmem_st32(tS + cc * 32, v);
+      }
+      ok = mbar_wait(&bars->dp_full, it & 1, 42);
+      if (ok && it > 0) ok = mbar_wait(&bars->ds_free, (it - 1) & 1, 43);
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int cc = 0; cc < BM / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tDP + cc * 32, v);
+        tmem_wait_ld();
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int c0 = cc * 32 + 2 * e;
+          const float d0 = pr[c0] * (__uint_as_float(v[2 * e]) - dsv[c0]);
+          const float d1 = pr[c0 + 1] * (__uint_as_float(v[2 * e + 1]) - dsv[c0 + 1]);
+          w[e] = pack_bf16x2(d0, d1);
+        }
+        // row r of the dS^T tile in the 128-byte swizzled layout: chunk cc/2,
+        // 16-byte units (cc%2)*4 .. +3 XOR (r % 8)
+        const uint32_t base = ds_row + (cc / 2) * C::CHUNK;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t unit = (uint32_t)((cc % 2) * 4 + u) ^ (uint32_t)(r & 7);
+          st_shared_v4(base + unit * 16, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars->ds_full);
+    }
+    if (ok) ok = mbar_wait(&bars->all_done, 0, 44);
+    if (ok) {
+      tc_fence_after();
+      const size_t row = (size_t)bh * p.N + (size_t)(key_ok ? kr : 0);
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tsrc = tmem + lane_off + (which ? C::T_DV : C::T_DK);
+        __nv_bfloat16* dst = (which ? p.dv : p.dk) + row * D;
+        const float mul = which ? 1.f : p.scale;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tsrc + cc * 32, v);
+          tmem_wait_ld();
+          if (key_ok) {
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              w[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+            uint4* o4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) o4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+          }
+        }
+      }
+    }
+  } else if (warp < 8) {
+    // dQ reduce group: query row r of each query tile
+    const int r = (warp % 4) * 32 + lane;
+    const uint32_t tQ = tmem + ((uint32_t)((warp % 4) * 32) << 16) + C::T_DP;
+    bool ok = true;
+    for (int it = 0; it < niter && ok; ++it) {
+      const int q = (i0 + it) * BM + r;
+      ok = mbar_wait(&bars->dq_full, it & 1, 45);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t v[D];
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tQ + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(v + cc * 32));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars->dq_empty);
+      if (q < p.N) {
+        float* dst = p.dq_acc + ((size_t)bh * p.N + q) * D;
+#pragma unroll
+        for (int g = 0; g < D / 4; ++g)
+          red_add_v4(dst + 4 * g, __uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
+                     __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// D, LSE*log2(e) (padded) and a zeroed dQ accumulator; one warp per padded row.
+template <int D>
+__global__ void __launch_bounds__(256) preprocess_kernel(const __nv_bfloat16* __restrict__ o,
+                                                         const __nv_bfloat16* __restrict__ dout,
+                                                         const float* __restrict__ lse,
+                                                         float* __restrict__ lse2,
+                                                         float* __restrict__ dsum,
+                                                         float* __restrict__ dq_acc, int BH, int N,
+                                                         int Npad) {
+  const long long gw = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (gw >= (long long)BH * Npad) return;
+  const int bh = (int)(gw / Npad), row = (int)(gw % Npad);
+  if (row >= N) {
+    if (lane == 0) {
+      lse2[gw] = INFINITY;
+      dsum[gw] = 0.f;
+    }
+    return;
+  }
+  const size_t off = ((size_t)bh * N + row) * D;
+  float acc = 0.f;
+#pragma unroll
+  for (int c = lane * 2; c < D; c += 64) {
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(o + off + c);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(dout + off + c);
+    acc = fmaf(__low2float(a), __low2float(b), acc);
+    acc = fmaf(__high2float(a), __high2float(b), acc);
+  }
+#pragma unroll
+  for (int sh = 16; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+  float4* z = reinterpret_cast<float4*>(dq_acc + off);
+  for (int c = lane; c < D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (lane == 0) {
+    dsum[gw] = acc;
+    lse2[gw] = lse[(size_t)bh * N + row] * kLog2e;
+  }
+}
+
+__global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict__ acc,
+                                                         __nv_bfloat16* __restrict__ dq, long long n4,
+                                                         float scale) {
+  for (long long idx = (long long)blockIdx.x * 256 + threadIdx.x; idx < n4;
+       idx += (long long)gridDim.x * 256) {
+    const float4 a = reinterpret_cast<const float4*>(acc)[idx];
+    uint2 w;
+    w.x = pack_bf16x2(a.x * scale, a.y * scale);
+    w.y = pack_bf16x2(a.z * scale, a.w * scale);
+    reinterpret_cast<uint2*>(dq)[idx] = w;
+  }
+}
+
+}  // namespace bwd
+
+size_t sm100_backward_workspace(int BH, int N, int d) {
+  const size_t npad = (size_t)(N + 127) / 128 * 128;
+  const size_t vec = ((size_t)BH * npad * 4 + 255) / 256 * 256;
+  const size_t acc = ((size_t)BH * N * d * 4 + 255) / 256 * 256;
+  return 2 * vec + acc;
+}
+
+cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                           const CUtensorMap& mdo, const void* o, const void* dout, const float* lse,
+                           void* dq, void* dk, void* dv, void* workspace, int BH, int N, int d,
+                           float scale, int causal, cudaStream_t st) {
+  const int npad = (N + 127) / 128 * 128;
+  const size_t vec = ((size_t)BH * npad * 4 + 255) / 256 * 256;
+  float* lse2 = static_cast<float*>(workspace);
+  float* dsum = reinterpret_cast<float*>(static_cast<char*>(workspace) + vec);
+  float* acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * vec);
+  const long long rows = (long long)BH * npad;
+  const unsigned pblocks = (unsigned)((rows + 7) / 8);
+  if (d == 128)
+    bwd::preprocess_kernel<128><<<pblocks, 256, 0, st>>>(
+        (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, lse2, dsum, acc, BH, N, npad);
+  else
+    bwd::preprocess_kernel<64><<<pblocks, 256, 0, st>>>(
+        (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, lse2, dsum, acc, BH, N, npad);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  bwd::Params p;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.dq_acc = acc;
+  p.lse2 = lse2;
+  p.dsum = dsum;
+  p.BH = BH;
+  p.N = N;
+  p.Npad = npad;
+  p.nkv = npad / 128;
+  p.scale = scale;
+  p.scale_log2 = scale * bwd::kLog2e;
+  p.causal = causal;
+  const dim3 grid((unsigned)(p.nkv * BH));
+  if (d == 128) {
+    const int smem = bwd::Cfg<128>::SMEM_BYTES;
+    e = cudaFuncSetAttribute(bwd::main_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    bwd::main_kernel<128><<<grid, bwd::NTHREADS, smem, st>>>(mq, mk, mv, mdo, p);
+  } else {
+    const int smem = bwd::Cfg<64>::SMEM_BYTES;
+    e = cudaFuncSetAttribute(bwd::main_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    bwd::main_kernel<64><<<grid, bwd::NTHREADS, smem, st>>>(mq, mk, mv, mdo, p);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long n4 = (long long)BH * N * d / 4;
+  const unsigned cblocks = (unsigned)std::min<long long>((n4 + 255) / 256, 148LL * 16);
+  bwd::dq_convert_kernel<<<cblocks, 256, 0, st>>>(acc, static_cast<__nv_bfloat16*>(dq), n4, scale);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

@@ -21,4 +21,12 @@ cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CU
                           void* o, float* lse, int BH, int N, int d, float scale, int causal,
                           cudaStream_t st);
 
+// tcgen05 backward (fa_bwd_sm100.cu): preprocess, main and dQ-convert kernels.
+// Workspace layout: LSE*log2(e) [BH, Npad], D [BH, Npad], fp32 dQ [BH, N, d].
+size_t sm100_backward_workspace(int BH, int N, int d);
+cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                           const CUtensorMap& mdo, const void* o, const void* dout, const float* lse,
+                           void* dq, void* dk, void* dv, void* workspace, int BH, int N, int d,
+                           float scale, int causal, cudaStream_t st);
+
 }  // namespace fa
