@@ -17,7 +17,7 @@ import os
 
 import torch
 
-__all__ = ["forward", "backward", "FAError", "library_path", "load_library", "check_device_status",
+__all__ = ["forward", "backward", "backward_noalloc", "FAError", "library_path", "load_library", "check_device_status",
            "workspace_size", "SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -31,6 +31,7 @@ SYMBOLS = {
     "fa_backward_workspace_size": (_Z, [_I, _I, _I, _I]),
     "fa_backward": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_fp32": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_backward_noalloc": (_I, [_P] * 9 + [_I, _I, _I, _I, _F, _I, _P]),
     "fa_check_device_status": (_I, [_P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
 }
@@ -145,6 +146,20 @@ def backward(q, k, v, o, do, lse, causal=False, scale=None, dq=None, dk=None, dv
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
               _ptr(workspace), workspace.numel() * workspace.element_size(), B, H, N, d, scale,
               int(bool(causal)), _stream(q)), "fa_backward")
+    return dq, dk, dv
+
+
+def backward_noalloc(q, k, v, o, do, lse, causal=False, scale=None, dq=None, dk=None, dv=None):
+    """dQ, dK, dV via fa_backward_noalloc: no workspace, the library's fixed scratch array."""
+    B, H, N, d = _shape(q)
+    _require((q, k, v, o, do), torch.bfloat16, (B, H, N, d))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(load_library().fa_backward_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv),
+        B, H, N, d, scale, int(bool(causal)), _stream(q)), "fa_backward_noalloc")
     return dq, dk, dv
 
 

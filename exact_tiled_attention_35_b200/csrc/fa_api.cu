@@ -188,3 +188,54 @@ const char* fa_status_string(fa_status status) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------
+// Allocation-free backward: the scratch of fa_backward in a fixed device
+// array.  Host code must not pass the array's name to a kernel (on the host it
+// names a stand-in, not device memory); its device address is looked up once
+// per device with cudaGetSymbolAddress while that device is current.
+
+namespace fa {
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_BACKWARD_NOALLOC_MAX_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (nullptr on error).
+void* noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  return g_noalloc_ptr[dev];
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" fa_status fa_backward_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                         const void* dout, const float* lse, void* dq, void* dk,
+                                         void* dv, int B, int H, int N, int d, float scale,
+                                         int causal, void* stream) {
+  fa_status s = check_shape(B, H, N, d, scale);
+  if (s != FA_OK) return s;
+  if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv})) != FA_OK) return s;
+  if (ws_bytes_for(B, H, N, d) > FA_BACKWARD_NOALLOC_MAX_BYTES) return FA_ERR_WORKSPACE;
+  if ((s = check_device()) != FA_OK) return s;
+  void* scratch = noalloc_scratch();
+  if (scratch == nullptr) return FA_ERR_CUDA;
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map(&mq, q, d, N, BH) || !make_map(&mk, k, d, N, BH) || !make_map(&mv, v, d, N, BH) ||
+      !make_map(&mdo, dout, d, N, BH))
+    return FA_ERR_CUDA;
+  return from_cuda(sm100_backward(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, scratch, BH, N, d,
+                                  scale, causal ? 1 : 0, static_cast<cudaStream_t>(stream)));
+}

@@ -89,6 +89,28 @@ fa_status fa_backward_fp32(const float* q, const float* k, const float* v, const
                            void* workspace, size_t ws_bytes, int B, int H, int N, int d,
                            float scale, int causal, void* stream);
 
+/* Largest scratch fa_backward_noalloc can use: 64 MiB, a fixed array inside the
+ * library that every GPU which loads the library keeps until process exit. */
+#define FA_BACKWARD_NOALLOC_MAX_BYTES ((size_t)64 << 20)
+
+/* Backward pass like fa_backward, for callers that cannot allocate device
+ * memory: for example a plug-in that only ever receives the input and output
+ * buffers of a host framework which owns all device memory, or a caller that
+ * must not issue cudaMalloc/cudaFree because those calls can synchronise the
+ * whole device and stall other work.  Same arguments, layout and results as
+ * fa_backward minus the workspace: the scratch lives in a fixed device array
+ * inside the library (FA_BACKWARD_NOALLOC_MAX_BYTES), so this call allocates
+ * nothing.  Shapes whose scratch (fa_backward_workspace_size) exceeds that
+ * limit return FA_ERR_WORKSPACE.  The first call on a device looks up the
+ * array's device address on that device (make it before any stream capture).
+ * All calls share the one array and the kernels re-initialise what they read,
+ * but two calls whose work overlaps on the GPU (different streams, no ordering
+ * between them) race on it.  The pages have no counterpart to this entry
+ * point; it exists only for callers without an allocator. */
+fa_status fa_backward_noalloc(const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                              int B, int H, int N, int d, float scale, int causal, void* stream);
+
 /* Synchronises `stream`, then reads and clears the current device's status
  * word.  FA_ERR_DEVICE_TIMEOUT if a kernel gave up a wait since the last call;
  * FA_ERR_CUDA if synchronisation failed; FA_OK otherwise. */
