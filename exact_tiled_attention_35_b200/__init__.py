@@ -33,6 +33,7 @@ SYMBOLS = {
     "fa_backward_fp32": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_noalloc": (_I, [_P] * 9 + [_I, _I, _I, _I, _F, _I, _P]),
     "fa_check_device_status": (_I, [_P]),
+    "fa_last_error": (ctypes.c_char_p, []),
     "fa_status_string": (ctypes.c_char_p, [_I]),
 }
 
@@ -42,7 +43,10 @@ class FAError(RuntimeError):
 
     def __init__(self, code, where):
         self.code = code
-        super().__init__(f"{where}: {status_string(code)} (fa_status {code})")
+        detail = ""
+        if code == 5:  # FA_ERR_CUDA
+            detail = ": " + load_library().fa_last_error().decode()
+        super().__init__(f"{where}: {status_string(code)}{detail} (fa_status {code})")
 
 
 def library_path():

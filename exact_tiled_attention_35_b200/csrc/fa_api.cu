@@ -91,7 +91,18 @@ fa_status check_device() {
   return FA_OK;
 }
 
-fa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+thread_local const char* g_last_error = "no error";
+
+fa_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return FA_OK;
+  g_last_error = cudaGetErrorString(e);
+  return FA_ERR_CUDA;
+}
+
+fa_status map_failed() {
+  g_last_error = "cuTensorMapEncodeTiled rejected a tensor map";
+  return FA_ERR_CUDA;
+}
 
 }  // namespace
 }  // namespace fa
@@ -109,7 +120,7 @@ fa_status fa_forward(const void* q, const void* k, const void* v, void* o, float
   const int BH = B * H;
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q, d, N, BH) || !make_map(&mk, k, d, N, BH) || !make_map(&mv, v, d, N, BH))
-    return FA_ERR_CUDA;
+    return map_failed();
   return from_cuda(sm100_forward(mq, mk, mv, o, lse, BH, N, d, scale, causal ? 1 : 0,
                                  static_cast<cudaStream_t>(stream)));
 }
@@ -142,7 +153,7 @@ fa_status fa_backward(const void* q, const void* k, const void* v, const void* o
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, q, d, N, BH) || !make_map(&mk, k, d, N, BH) || !make_map(&mv, v, d, N, BH) ||
       !make_map(&mdo, dout, d, N, BH))
-    return FA_ERR_CUDA;
+    return map_failed();
   return from_cuda(sm100_backward(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, workspace, BH, N, d,
                                   scale, causal ? 1 : 0, static_cast<cudaStream_t>(stream)));
 }
@@ -173,6 +184,8 @@ fa_status fa_check_device_status(void* stream) {
     return FA_ERR_CUDA;
   return word ? FA_ERR_DEVICE_TIMEOUT : FA_OK;
 }
+
+const char* fa_last_error(void) { return g_last_error; }
 
 const char* fa_status_string(fa_status status) {
   switch (status) {
@@ -235,7 +248,7 @@ extern "C" fa_status fa_backward_noalloc(const void* q, const void* k, const voi
   CUtensorMap mq, mk, mv, mdo;
   if (!make_map(&mq, q, d, N, BH) || !make_map(&mk, k, d, N, BH) || !make_map(&mv, v, d, N, BH) ||
       !make_map(&mdo, dout, d, N, BH))
-    return FA_ERR_CUDA;
+    return map_failed();
   return from_cuda(sm100_backward(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, scratch, BH, N, d,
                                   scale, causal ? 1 : 0, static_cast<cudaStream_t>(stream)));
 }

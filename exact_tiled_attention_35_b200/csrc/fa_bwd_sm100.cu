@@ -19,12 +19,14 @@
 //   convert     dQ = scale * accumulator, rounded to bf16.
 //
 // Main-kernel CTA layout (320 threads):
-//   warps 0-3  P / dS computation (thread = key row = tensor-memory lane),
-//              then the dK / dV epilogue
-//   warps 4-7  dQ reduce: tensor memory -> registers -> red.global.add.v4.f32
+//   warps 0-7  P / dS computation (thread = key row = tensor-memory lane, two
+//              warps per row quarter, one per half of the query columns), the
+//              dQ drain (tensor memory -> registers -> red.global.add.v4.f32)
+//              and the dK / dV epilogue
 //   warp  8    TMA producer: K, V once; Q_i, dO_i, LSE_i, D_i per query tile
 //   warp  9    tensor-memory allocator and MMA issuer
-// Tensor memory: S^T / P^T at column 0, dP^T / dQ at 128, dV at 256, dK at 256+d.
+// Tensor memory: S^T at column 0 (P^T of query columns 64h.. packed at column 64h),
+// dP^T / dQ at 128, dV at 256, dK at 256+d.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -87,6 +89,7 @@ struct Bars {
   uint64_t qdo_empty[NST];
   uint64_t s_full;
   uint64_t dp_full;
+  uint64_t p_full;
   uint64_t ds_full;
   uint64_t ds_free;
   uint64_t dq_full;
@@ -112,6 +115,39 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ float4 ld_shared_v4(uint32_t addr) {
+  float4 r;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+               : "r"(addr));
+  return r;
+}
+
+// In-warp transpose of 8x8 blocks of 4 floats inside each group of 8 lanes:
+// on entry lane 8a+b holds row 8a+b, column blocks 0..7 (x[s] = columns 4s..4s+3);
+// on exit it holds column block b of rows 8a+0 .. 8a+7 (x[s] = row 8a+s).  Three
+// butterfly stages; in the stage for bit m, lanes with bit m set swap the
+// blocks whose index has bit m clear with their partner lane (lane ^ m).
+__device__ __forceinline__ void transpose8x8x4(float (&x)[8][4], int lane) {
+#pragma unroll
+  for (int m = 4; m >= 1; m >>= 1) {
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      if (s & m) continue;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float send = upper ? x[s][e] : x[s | m][e];
+        const float recv = __shfl_xor_sync(0xffffffffu, send, m);
+        if (upper)
+          x[s][e] = recv;
+        else
+          x[s | m][e] = recv;
+      }
+    }
+  }
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
@@ -157,10 +193,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->ds_full, 128);
+    mbar_init(&bars->p_full, 2 * 128);
+    mbar_init(&bars->ds_full, 2 * 128);
     mbar_init(&bars->ds_free, 1);
     mbar_init(&bars->dq_full, 1);
-    mbar_init(&bars->dq_empty, 128);
+    mbar_init(&bars->dq_empty, 2 * 128);
     mbar_init(&bars->all_done, 1);
     mbar_init(&bars->drain, 1);
     fence_mbar_init();
@@ -245,6 +282,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  C::IDESC_S, kk > 0);
         }
         mma_commit(&bars->dp_full);
+        ok = mbar_wait(&bars->p_full, it & 1, 46);
+        if (!ok) break;
+        tc_fence_after();
+        // dV += P^T dO  (keys x d), K = 128 queries, P^T from tensor memory (queries
+        // 64h .. 64h+63 packed at column 64h); runs while the compute warps form dS
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_ts(tmem + C::T_DV, tmem + C::T_S + 64 * (kk / 4) + 8 * (kk % 4),
+                 sdesc_sw128(udO + kk * 2048, C::CHUNK, 1024),
+                 C::IDESC_DKV, (it > 0 || kk > 0) ? 1u : 0u);
         ok = mbar_wait(&bars->ds_full, it & 1, 38);
         if (!ok) break;
         tc_fence_after();
@@ -254,11 +301,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mma_ss(tmem + C::T_DP, sdesc_sw128(uDS + kk * 2048, C::CHUNK, 1024),
                  sdesc_sw128(uK + kk * 2048, C::CHUNK, 1024), C::IDESC_DQ, kk > 0);
         mma_commit(&bars->dq_full);
-        // dV += P^T dO  (keys x d), K = 128 queries, P^T from tensor memory
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ts(tmem + C::T_DV, tmem + C::T_S + kk * 8, sdesc_sw128(udO + kk * 2048, C::CHUNK, 1024),
-                 C::IDESC_DKV, (it > 0 || kk > 0) ? 1u : 0u);
         // dK += dS^T Q  (keys x d), K = 128 queries
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
@@ -274,84 +316,126 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mma_commit(&bars->drain);
       mbar_wait(&bars->drain, 0, 39);
     }
-  } else if (warp < 4) {
-    // P^T and dS for key row r of this tile
-    const int r = warp * 32 + lane;
+  } else {
+    // Compute warps 0-7.  Warp w owns tensor-memory lane quarter w % 4 (key rows
+    // 32*(w%4) .. +31 for S^T/dP^T/dK/dV, query rows for dQ) and column half
+    // h = w / 4: query columns 64h .. 64h+63 of P^T and dS, dQ / dK / dV columns
+    // (d/2)h .. (d/2)h + d/2 - 1.  Per query tile: P^T -> tensor memory, dS ->
+    // shared memory, then the partial dQ of the tile is drained from tensor memory
+    // and added to the fp32 accumulator while the tensor core runs dK and the next
+    // tile's S^T and dP^T.
+    const int qw = warp % 4, h = warp / 4;
+    const int r = qw * 32 + lane;
     const int kr = j * BN + r;
     const bool key_ok = kr < p.N;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::T_S;
     const uint32_t tDP = tmem + lane_off + C::T_DP;
     const float c = p.scale_log2;
-    const uint32_t ds_row = smem_u32(sDS) + r * 128;
+    const uint32_t ds_row = smem_u32(sDS) + h * C::CHUNK + r * 128;
+    const int grp = lane >> 3, blk = lane & 7;
+    constexpr int DH = D / 2;  // dQ / dK / dV columns per warp
     bool ok = true;
     for (int it = 0; it < niter && ok; ++it) {
       const int i = i0 + it, st = it % NST;
-      const float* lse2 = sVec + st * 2 * BM;
-      const float* dsv = lse2 + BM;
+      const uint32_t lse2 = smem_u32(sVec + st * 2 * BM) + h * 64 * 4;  // LSE*log2(e), my columns
+      const uint32_t dsv = lse2 + BM * 4;                                // D, my columns
       ok = mbar_wait(&bars->qdo_full[st], (it / NST) & 1, 40);
       if (ok) ok = mbar_wait(&bars->s_full, it & 1, 41);
       if (!ok) break;
       tc_fence_after();
-      float pr[BM];
+      float pr[64];
 #pragma unroll
-      for (int cc = 0; cc < BM / 32; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t v[32];
-        tmem_ld32(tS + cc * 32, v);
+        tmem_ld32(tS + h * 64 + cc * 32, v);
 #pragma unroll
         for (int e = 0; e < 32; ++e) pr[cc * 32 + e] = __uint_as_float(v[e]);
       }
       tmem_wait_ld();
       const bool diag = p.causal && i == j;
 #pragma unroll
-      for (int c4 = 0; c4 < BM / 4; ++c4) {
-        const float4 l4 = reinterpret_cast<const float4*>(lse2)[c4];
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 l4 = ld_shared_v4(lse2 + c4 * 16);
         const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int col = c4 * 4 + e;
           float pv = ex2(fmaf(pr[col], c, -lv[e]));
-          if (!key_ok || (diag && col < r)) pv = 0.f;
+          if (!key_ok || (diag && h * 64 + col < r)) pv = 0.f;
           pr[col] = pv;
         }
       }
-#pragma unroll
-      for (int cc = 0; cc < BM / 64; ++cc) {
+      {
         uint32_t v[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = pack_bf16x2(pr[cc * 64 + 2 * e], pr[cc * 64 + 2 * e + 1]);
-        tmem_st32(tS + cc * 32, v);
+        for (int e = 0; e < 32; ++e) v[e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
+        // packed P^T of my 64 query columns over the first 32 of my own S columns
+        tmem_st32(tS + h * 64, v);
       }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full);
       ok = mbar_wait(&bars->dp_full, it & 1, 42);
       if (ok && it > 0) ok = mbar_wait(&bars->ds_free, (it - 1) & 1, 43);
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < BM / 32; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         uint32_t v[32];
-        tmem_ld32(tDP + cc * 32, v);
+        tmem_ld32(tDP + h * 64 + cc * 32, v);
         tmem_wait_ld();
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c0 = cc * 32 + 2 * e;
-          const float d0 = pr[c0] * (__uint_as_float(v[2 * e]) - dsv[c0]);
-          const float d1 = pr[c0 + 1] * (__uint_as_float(v[2 * e + 1]) - dsv[c0 + 1]);
-          w[e] = pack_bf16x2(d0, d1);
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const int c0 = cc * 32 + 4 * e4;
+          const float4 dd = ld_shared_v4(dsv + c0 * 4);
+          w[2 * e4] = pack_bf16x2(pr[c0] * (__uint_as_float(v[4 * e4]) - dd.x),
+                                  pr[c0 + 1] * (__uint_as_float(v[4 * e4 + 1]) - dd.y));
+          w[2 * e4 + 1] = pack_bf16x2(pr[c0 + 2] * (__uint_as_float(v[4 * e4 + 2]) - dd.z),
+                                      pr[c0 + 3] * (__uint_as_float(v[4 * e4 + 3]) - dd.w));
         }
-        // row r of the dS^T tile in the 128-byte swizzled layout: chunk cc/2,
-        // 16-byte units (cc%2)*4 .. +3 XOR (r % 8)
-        const uint32_t base = ds_row + (cc / 2) * C::CHUNK;
+        // row r of the dS^T tile in the 128-byte swizzled layout: chunk h,
+        // 16-byte units cc*4 .. cc*4+3 XOR (r % 8)
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const uint32_t unit = (uint32_t)((cc % 2) * 4 + u) ^ (uint32_t)(r & 7);
-          st_shared_v4(base + unit * 16, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+          const uint32_t unit = (uint32_t)(cc * 4 + u) ^ (uint32_t)(r & 7);
+          st_shared_v4(ds_row + unit * 16, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
         }
       }
-      tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars->ds_full);
+      // drain the partial dQ of this tile: rows = queries of tile i
+      ok = mbar_wait(&bars->dq_full, it & 1, 45);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t q[DH];
+#pragma unroll
+      for (int cc = 0; cc < DH / 32; ++cc)
+        tmem_ld32(tDP + h * DH + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(q + cc * 32));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars->dq_empty);
+      // transpose each 32-column chunk inside groups of 8 lanes so that one
+      // red.global.add.v4 covers 4 query rows x 128 contiguous bytes
+      const int row0 = i * BM + qw * 32 + grp * 8;
+#pragma unroll
+      for (int cc = 0; cc < DH / 32; ++cc) {
+        float x[8][4];
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[s][e] = __uint_as_float(q[cc * 32 + 4 * s + e]);
+        transpose8x8x4(x, lane);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const int qrow = row0 + s;
+          if (qrow < p.N)
+            red_add_v4(p.dq_acc + ((size_t)bh * p.N + qrow) * D + h * DH + cc * 32 + 4 * blk,
+                       x[s][0], x[s][1], x[s][2], x[s][3]);
+        }
+      }
     }
     if (ok) ok = mbar_wait(&bars->all_done, 0, 44);
     if (ok) {
@@ -359,11 +443,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const size_t row = (size_t)bh * p.N + (size_t)(key_ok ? kr : 0);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
-        const uint32_t tsrc = tmem + lane_off + (which ? C::T_DV : C::T_DK);
-        __nv_bfloat16* dst = (which ? p.dv : p.dk) + row * D;
+        const uint32_t tsrc = tmem + lane_off + (which ? C::T_DV : C::T_DK) + h * DH;
+        __nv_bfloat16* dst = (which ? p.dv : p.dk) + row * D + h * DH;
         const float mul = which ? 1.f : p.scale;
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
+        for (int cc = 0; cc < DH / 32; ++cc) {
           uint32_t v[32];
           tmem_ld32(tsrc + cc * 32, v);
           tmem_wait_ld();
@@ -377,30 +461,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int u = 0; u < 4; ++u) o4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
           }
         }
-      }
-    }
-  } else if (warp < 8) {
-    // dQ reduce group: query row r of each query tile
-    const int r = (warp % 4) * 32 + lane;
-    const uint32_t tQ = tmem + ((uint32_t)((warp % 4) * 32) << 16) + C::T_DP;
-    bool ok = true;
-    for (int it = 0; it < niter && ok; ++it) {
-      const int q = (i0 + it) * BM + r;
-      ok = mbar_wait(&bars->dq_full, it & 1, 45);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t v[D];
-#pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tQ + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(v + cc * 32));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bars->dq_empty);
-      if (q < p.N) {
-        float* dst = p.dq_acc + ((size_t)bh * p.N + q) * D;
-#pragma unroll
-        for (int g = 0; g < D / 4; ++g)
-          red_add_v4(dst + 4 * g, __uint_as_float(v[4 * g]), __uint_as_float(v[4 * g + 1]),
-                     __uint_as_float(v[4 * g + 2]), __uint_as_float(v[4 * g + 3]));
       }
     }
   }

@@ -116,6 +116,11 @@ fa_status fa_backward_noalloc(const void* q, const void* k, const void* v, const
  * FA_ERR_CUDA if synchronisation failed; FA_OK otherwise. */
 fa_status fa_check_device_status(void* stream);
 
+/* Text of the most recent CUDA error that an fa_* call on the calling thread
+ * ran into (after FA_ERR_CUDA), or "no error".  Valid until the next fa_* call
+ * on the same thread. */
+const char* fa_last_error(void);
+
 /* Static, NUL-terminated description of a status code. */
 const char* fa_status_string(fa_status status);
 
