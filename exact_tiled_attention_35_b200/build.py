@@ -10,7 +10,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfa.so")
-SOURCES = ["fa_api.cu", "fa_simt.cu", "fa_fwd_sm100.cu", "fa_bwd_sm100.cu"]
+SOURCES = ["fa_lib.cu"]  # includes fa_api.cu, fa_simt.cu, fa_fwd_sm100.cu, fa_bwd_sm100.cu
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 
@@ -31,7 +31,7 @@ def build(force=False, verbose=False):
     if not force and up_to_date():
         return LIB
     cmd = [
-        NVCC, "-shared", "-Xcompiler", "-fPIC", "-rdc=true",
+        NVCC, "-shared", "-Xcompiler", "-fPIC",
         "-gencode", "arch=compute_100a,code=sm_100a",
         "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
         "-I", os.path.join(os.path.dirname(HERE), "include"),

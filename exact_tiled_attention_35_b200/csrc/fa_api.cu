@@ -17,7 +17,7 @@
 
 namespace fa {
 
-__device__ unsigned int g_device_status = 0;
+// the device status word g_device_status is defined in fa_device.cuh
 
 namespace {
 

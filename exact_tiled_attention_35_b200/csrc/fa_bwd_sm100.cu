@@ -18,13 +18,13 @@
 //               the fp32 accumulator with vector atomics;
 //   convert     dQ = scale * accumulator, rounded to bf16.
 //
-// Main-kernel CTA layout (320 threads):
-//   warps 0-7  P / dS computation (thread = key row = tensor-memory lane, two
-//              warps per row quarter, one per half of the query columns), the
-//              dQ drain (tensor memory -> registers -> red.global.add.v4.f32)
-//              and the dK / dV epilogue
-//   warp  8    TMA producer: K, V once; Q_i, dO_i, LSE_i, D_i per query tile
-//   warp  9    tensor-memory allocator and MMA issuer
+// Main-kernel CTA layout (512 threads, registers rebalanced with setmaxnreg):
+//   warps 0-7   P / dS computation (thread = key row = tensor-memory lane, two
+//               warps per row quarter, one per half of the query columns) and
+//               the dK / dV epilogue
+//   warps 8-11  dQ drain: tensor memory -> registers -> red.global.add.v4.f32
+//   warp  12    TMA producer: K, V once; Q_i, dO_i, LSE_i, D_i per query tile
+//   warp  13    tensor-memory allocator and MMA issuer (warps 14-15 idle)
 // Tensor memory: S^T at column 0 (P^T of query columns 64h.. packed at column 64h),
 // dP^T / dQ at 128, dV at 256, dK at 256+d.
 
@@ -44,9 +44,17 @@ namespace bwd {
 
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per tile
-constexpr int NTHREADS = 320;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int NTHREADS = 512;     // four warpgroups
+constexpr int kProducerWarp = 12;
+constexpr int kMmaWarp = 13;
+// Register split (setmaxnreg).  The launch gives every thread 128 registers,
+// 512 * 128 = 65536 in all; the shares below sum to 128 * (2*144 + 144 + 80) =
+// 65536, exactly that pool.
+constexpr int kRegsCompute = 144;  // warpgroups 0 and 1
+constexpr int kRegsReduce = 144;   // warpgroup 2
+constexpr int kRegsControl = 80;   // warpgroup 3: producer, MMA issuer, two idle warps
+static_assert(128 * (2 * kRegsCompute + kRegsReduce + kRegsControl) <= 512 * 128,
+              "register split exceeds the launch allocation");
 constexpr int NST = 2;  // Q / dO stages
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -197,7 +205,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&bars->ds_full, 2 * 128);
     mbar_init(&bars->ds_free, 1);
     mbar_init(&bars->dq_full, 1);
-    mbar_init(&bars->dq_empty, 2 * 128);
+    mbar_init(&bars->dq_empty, 128);
     mbar_init(&bars->all_done, 1);
     mbar_init(&bars->drain, 1);
     fence_mbar_init();
@@ -217,7 +225,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == kProducerWarp) {
+  if (warp >= 12) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
+   if (warp == kProducerWarp) {
     if (lane == 0) {
       mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
       for (int c = 0; c < D / 64; ++c) {
@@ -250,7 +260,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_wait(&bars->qdo_full[s], (last / NST) & 1, 34);
       }
     }
-  } else if (warp == kMmaWarp) {
+   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       const uint32_t uK = smem_u32(sK), uV = smem_u32(sV), uDS = smem_u32(sDS);
       bool ok = mbar_wait(&bars->kv_full, 0, 35);
@@ -316,7 +326,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mma_commit(&bars->drain);
       mbar_wait(&bars->drain, 0, 39);
     }
-  } else {
+   }
+  } else if (warp < 8) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsCompute));
     // Compute warps 0-7.  Warp w owns tensor-memory lane quarter w % 4 (key rows
     // 32*(w%4) .. +31 for S^T/dP^T/dK/dV, query rows for dQ) and column half
     // h = w / 4: query columns 64h .. 64h+63 of P^T and dS, dQ / dK / dV columns
@@ -333,7 +345,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tDP = tmem + lane_off + C::T_DP;
     const float c = p.scale_log2;
     const uint32_t ds_row = smem_u32(sDS) + h * C::CHUNK + r * 128;
-    const int grp = lane >> 3, blk = lane & 7;
     constexpr int DH = D / 2;  // dQ / dK / dV columns per warp
     bool ok = true;
     for (int it = 0; it < niter && ok; ++it) {
@@ -406,36 +417,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&bars->ds_full);
-      // drain the partial dQ of this tile: rows = queries of tile i
-      ok = mbar_wait(&bars->dq_full, it & 1, 45);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t q[DH];
-#pragma unroll
-      for (int cc = 0; cc < DH / 32; ++cc)
-        tmem_ld32(tDP + h * DH + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(q + cc * 32));
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bars->dq_empty);
-      // transpose each 32-column chunk inside groups of 8 lanes so that one
-      // red.global.add.v4 covers 4 query rows x 128 contiguous bytes
-      const int row0 = i * BM + qw * 32 + grp * 8;
-#pragma unroll
-      for (int cc = 0; cc < DH / 32; ++cc) {
-        float x[8][4];
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) x[s][e] = __uint_as_float(q[cc * 32 + 4 * s + e]);
-        transpose8x8x4(x, lane);
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const int qrow = row0 + s;
-          if (qrow < p.N)
-            red_add_v4(p.dq_acc + ((size_t)bh * p.N + qrow) * D + h * DH + cc * 32 + 4 * blk,
-                       x[s][0], x[s][1], x[s][2], x[s][3]);
-        }
-      }
     }
     if (ok) ok = mbar_wait(&bars->all_done, 0, 44);
     if (ok) {
@@ -460,6 +441,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
             for (int u = 0; u < 4; ++u) o4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
           }
+        }
+      }
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsReduce));
+    // dQ reduce warps 8-11: warp w drains query rows 32*(w%4) .. +31 of each
+    // tile's partial dQ (all d columns) from tensor memory, then adds them to the
+    // fp32 accumulator.  Each 32-column chunk is transposed inside groups of 8
+    // lanes so that one red.global.add.v4 covers 4 rows x 128 contiguous bytes.
+    const int qw = warp % 4;
+    const uint32_t tQ = tmem + ((uint32_t)(qw * 32) << 16) + C::T_DP;
+    const int grp = lane >> 3, blk = lane & 7;
+    bool ok = true;
+    for (int it = 0; it < niter && ok; ++it) {
+      ok = mbar_wait(&bars->dq_full, it & 1, 45);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t q[D / 32][32];
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tQ + cc * 32, q[cc]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars->dq_empty);
+      const int row0 = (i0 + it) * BM + qw * 32 + grp * 8;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        float x[8][4];
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[s][e] = __uint_as_float(q[cc][4 * s + e]);
+        transpose8x8x4(x, lane);
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          const int qrow = row0 + s;
+          if (qrow < p.N)
+            red_add_v4(p.dq_acc + ((size_t)bh * p.N + qrow) * D + cc * 32 + 4 * blk, x[s][0],
+                       x[s][1], x[s][2], x[s][3]);
         }
       }
     }

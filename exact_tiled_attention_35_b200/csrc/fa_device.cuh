@@ -12,7 +12,7 @@ namespace fa {
 
 // Status word shared by every kernel in the library (one per device).  A kernel
 // whose bounded wait runs out stores a nonzero site code here and returns.
-extern __device__ unsigned int g_device_status;
+__device__ unsigned int g_device_status = 0;
 
 // A wait that has not finished after this many nanoseconds is treated as a hang.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
