@@ -22,7 +22,7 @@
 //   warps 0-7   P / dS computation (thread = key row = tensor-memory lane, two
 //               warps per row quarter, one per half of the query columns) and
 //               the dK / dV epilogue
-//   warps 8-11  dQ drain: tensor memory -> registers -> red.global.add.v4.f32
+//   warps 8-11  dQ drain: tensor memory -> registers -> red.global.add.v2.f32
 //   warp  12    TMA producer: K, V once; Q_i, dO_i, LSE_i, D_i per query tile
 //   warp  13    tensor-memory allocator and MMA issuer (warps 14-15 idle)
 // Tensor memory: S^T at column 0 (P^T of query columns 64h.. packed at column 64h),
@@ -48,11 +48,11 @@ constexpr int NTHREADS = 512;     // four warpgroups
 constexpr int kProducerWarp = 12;
 constexpr int kMmaWarp = 13;
 // Register split (setmaxnreg).  The launch gives every thread 128 registers,
-// 512 * 128 = 65536 in all; the shares below sum to 128 * (2*144 + 144 + 80) =
+// 512 * 128 = 65536 in all; the shares below sum to 128 * (2*144 + 136 + 88) =
 // 65536, exactly that pool.
 constexpr int kRegsCompute = 144;  // warpgroups 0 and 1
-constexpr int kRegsReduce = 144;   // warpgroup 2
-constexpr int kRegsControl = 80;   // warpgroup 3: producer, MMA issuer, two idle warps
+constexpr int kRegsReduce = 136;   // warpgroup 2
+constexpr int kRegsControl = 88;   // warpgroup 3: producer, MMA issuer, two idle warps
 static_assert(128 * (2 * kRegsCompute + kRegsReduce + kRegsControl) <= 512 * 128,
               "register split exceeds the launch allocation");
 constexpr int NST = 2;  // Q / dO stages
@@ -113,6 +113,10 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
+__device__ __forceinline__ void red_add_v2(float* addr, float a, float b) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(addr), "f"(a), "f"(b) : "memory");
+}
+
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -131,31 +135,6 @@ __device__ __forceinline__ float4 ld_shared_v4(uint32_t addr) {
                : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
                : "r"(addr));
   return r;
-}
-
-// In-warp transpose of 8x8 blocks of 4 floats inside each group of 8 lanes:
-// on entry lane 8a+b holds row 8a+b, column blocks 0..7 (x[s] = columns 4s..4s+3);
-// on exit it holds column block b of rows 8a+0 .. 8a+7 (x[s] = row 8a+s).  Three
-// butterfly stages; in the stage for bit m, lanes with bit m set swap the
-// blocks whose index has bit m clear with their partner lane (lane ^ m).
-__device__ __forceinline__ void transpose8x8x4(float (&x)[8][4], int lane) {
-#pragma unroll
-  for (int m = 4; m >= 1; m >>= 1) {
-    const bool upper = (lane & m) != 0;
-#pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      if (s & m) continue;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float send = upper ? x[s][e] : x[s | m][e];
-        const float recv = __shfl_xor_sync(0xffffffffu, send, m);
-        if (upper)
-          x[s][e] = recv;
-        else
-          x[s | m][e] = recv;
-      }
-    }
-  }
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
@@ -447,38 +426,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsReduce));
     // dQ reduce warps 8-11: warp w drains query rows 32*(w%4) .. +31 of each
-    // tile's partial dQ (all d columns) from tensor memory, then adds them to the
-    // fp32 accumulator.  Each 32-column chunk is transposed inside groups of 8
-    // lanes so that one red.global.add.v4 covers 4 rows x 128 contiguous bytes.
+    // tile's partial dQ from tensor memory and adds them to the fp32 accumulator.
+    // It reads 16 rows x 64 columns at a time in the 16x256b shape, where four
+    // adjacent lanes hold 8 contiguous columns of one row, so each
+    // red.global.add.v2 instruction covers 8 rows x 32 contiguous bytes.
     const int qw = warp % 4;
     const uint32_t tQ = tmem + ((uint32_t)(qw * 32) << 16) + C::T_DP;
-    const int grp = lane >> 3, blk = lane & 7;
     bool ok = true;
     for (int it = 0; it < niter && ok; ++it) {
       ok = mbar_wait(&bars->dq_full, it & 1, 45);
       if (!ok) break;
       tc_fence_after();
-      uint32_t q[D / 32][32];
+      const int tile_row = (i0 + it) * BM + qw * 32 + lane / 4;
+      constexpr int NPART = 2 * (D / 64);
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tQ + cc * 32, q[cc]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bars->dq_empty);
-      const int row0 = (i0 + it) * BM + qw * 32 + grp * 8;
+      for (int part = 0; part < NPART; ++part) {
+        const int hh = part / (D / 64), ch = part % (D / 64);  // lane half, 64-column block
+        uint32_t v[32];
+        tmem_ld16x256b_x8(tQ + ((uint32_t)(16 * hh) << 16) + ch * 64, v);
+        tmem_wait_ld();
+        if (part == NPART - 1) {
+          tc_fence_before();
+          mbar_arrive(&bars->dq_empty);
+        }
+        const int r0 = tile_row + 16 * hh, r1 = r0 + 8;
+        const int col = ch * 64 + 2 * (lane % 4);
+        float* d0 = p.dq_acc + ((size_t)bh * p.N + r0) * D + col;
+        float* d1 = p.dq_acc + ((size_t)bh * p.N + r1) * D + col;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        float x[8][4];
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) x[s][e] = __uint_as_float(q[cc][4 * s + e]);
-        transpose8x8x4(x, lane);
-#pragma unroll
-        for (int s = 0; s < 8; ++s) {
-          const int qrow = row0 + s;
-          if (qrow < p.N)
-            red_add_v4(p.dq_acc + ((size_t)bh * p.N + qrow) * D + cc * 32 + 4 * blk, x[s][0],
-                       x[s][1], x[s][2], x[s][3]);
+        for (int jb = 0; jb < 8; ++jb) {
+          if (r0 < p.N) red_add_v2(d0 + 8 * jb, __uint_as_float(v[4 * jb]), __uint_as_float(v[4 * jb + 1]));
+          if (r1 < p.N)
+            red_add_v2(d1 + 8 * jb, __uint_as_float(v[4 * jb + 2]), __uint_as_float(v[4 * jb + 3]));
         }
       }
     }

@@ -11,15 +11,18 @@
 // stays unnormalised until the last tile and is divided by l once.  Tile size
 // 128 follows the block size the nisoo.com page reports as typical.
 //
-// CTA layout (320 threads):
+// CTA layout (384 threads, registers rebalanced with setmaxnreg):
 //   warps 0-3  softmax + epilogue for query tile 0 (tensor-memory lanes 0-127)
 //   warps 4-7  softmax + epilogue for query tile 1
 //   warp  8    TMA producer: Q tiles once, then K_j, V_j into a ring of slots
 //   warp  9    tensor-memory allocator and MMA issuer (one elected thread)
+//   warps 10-11 idle (they complete the third warpgroup)
 // Tensor memory (512 columns): S_t at column 128*t (fp32 128x128, the bf16
 // probabilities P_t are written over its first 64 columns), O_t at 256 + D*t.
 // MMA order per key tile j: PV_0(j), S_0(j+1), PV_1(j), S_1(j+1), so while one
-// softmax group works on its scores the tensor core runs the other's GEMMs.
+// softmax group works on its scores the tensor core runs the other's GEMMs.  Each
+// P V is issued in two halves of 64 keys, as soon as the softmax group has
+// written that half of P.
 //
 // A row's maximum is only raised when it grows by more than 2^8 in the exp2
 // domain; P and l then use the same (stale) maximum, so O = O_acc / l and
@@ -41,9 +44,15 @@ namespace fwd {
 constexpr int BM = 128;           // query rows per tile
 constexpr int BN = 128;           // keys per tile
 constexpr int NQT = 2;            // query tiles per CTA
-constexpr int NTHREADS = 320;
+constexpr int NTHREADS = 384;  // three warpgroups
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+// Register split (setmaxnreg).  The launch gives every thread 168 registers,
+// 384 * 168 = 64512 in all; the shares sum to 128 * (2*208 + 88) = 64512.
+constexpr int kRegsSoftmax = 208;  // warpgroups 0 and 1
+constexpr int kRegsControl = 88;   // warpgroup 2: producer, MMA issuer, two idle warps
+static_assert(128 * (2 * kRegsSoftmax + kRegsControl) <= NTHREADS * 168,
+              "register split exceeds the launch allocation");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -75,7 +84,8 @@ struct Params {
 struct Bars {
   uint64_t q_full[NQT];
   uint64_t s_full[NQT];
-  uint64_t p_full[NQT];
+  uint64_t p_lo[NQT];   // probabilities of keys 0-63 of the tile in tensor memory
+  uint64_t p_hi[NQT];   // keys 64-127
   uint64_t o_full;
   uint64_t drain;
   uint64_t kv_full[16];
@@ -119,7 +129,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     for (int t = 0; t < NQT; ++t) {
       mbar_init(&bars->q_full[t], 1);
       mbar_init(&bars->s_full[t], 1);
-      mbar_init(&bars->p_full[t], 128);
+      mbar_init(&bars->p_lo[t], 128);
+      mbar_init(&bars->p_hi[t], 128);
     }
     mbar_init(&bars->o_full, 1);
     mbar_init(&bars->drain, 1);
@@ -143,7 +154,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  if (warp == kProducerWarp) {
+  if (warp >= 8) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
+   if (warp == kProducerWarp) {
     if (lane == 0) {
       bool ok = true;
       for (int t = 0; t < NQT; ++t) {
@@ -173,7 +186,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_wait(&bars->kv_full[s], (last / C::NSLOT) & 1, 2);
       }
     }
-  } else if (warp == kMmaWarp) {
+   } else if (warp == kMmaWarp) {
     if (lane == 0) {
       bool ok = true;
       const uint32_t sq = smem_u32(sQ), sr = smem_u32(sRing);
@@ -190,13 +203,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  C::IDESC_QK, kk > 0);
         }
       };
-      // O_t += P_t V_j : A = P_t (tensor memory), B = V_j (MN-major), K = 128 keys
-      auto issue_pv = [&](int t, int j) {
+      // O_t += P_t V_j : A = P_t (tensor memory), B = V_j (MN-major), K = 128 keys,
+      // issued in two halves (keys 0-63, 64-127) as the softmax group publishes them
+      auto issue_pv = [&](int t, int j, int half) {
         const uint32_t b0 = sr + slot_of(2 * j + 1) * C::TILE;
         const uint32_t d_tmem = tmem + 2 * BN + t * D;
         const uint32_t a_tmem = tmem + t * BN;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
+        for (int kk = half * 4; kk < half * 4 + 4; ++kk)
           mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b0 + kk * 16 * 128, C::CHUNK, 1024),
                  C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
       };
@@ -217,10 +231,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         bool k_next_ready = false;
         for (int t = 0; t < NQT && ok; ++t) {
           if (j >= ntile[t]) continue;
-          ok = mbar_wait(&bars->p_full[t], j & 1, 6);
+          ok = mbar_wait(&bars->p_lo[t], j & 1, 6);
           if (!ok) break;
           tc_fence_after();
-          issue_pv(t, j);
+          issue_pv(t, j, 0);
+          ok = mbar_wait(&bars->p_hi[t], j & 1, 9);
+          if (!ok) break;
+          tc_fence_after();
+          issue_pv(t, j, 1);
           if (j + 1 < ntile[t]) {
             if (!k_next_ready) {
               ok = mbar_wait(&bars->kv_full[slot_of(2 * j + 2)], phase_of(2 * j + 2), 7);
@@ -241,7 +259,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mma_commit(&bars->drain);
       mbar_wait(&bars->drain, 0, 8);
     }
+   }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
     // softmax / epilogue groups
     const int t = warp / 4;
     const int row = (warp % 4) * 32 + lane;
@@ -276,8 +296,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       float mx4[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-      for (int i = 4; i < BN; ++i) mx4[i % 4] = fmaxf(mx4[i % 4], s[i]);
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+      for (int i = 4; i < BN; i += 2) mx4[(i / 2) % 4] = fmax3(mx4[(i / 2) % 4], s[i], s[i + 1]);
+      const float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
       const float m_new = fmaxf(m_used, mx);
       const bool need = (m_new - m_used) * c > kRescaleThreshold;
       float alpha = 1.f;
@@ -285,18 +305,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         alpha = ex2((m_used - m_new) * c);
         m_used = m_new;
       }
-      // a row that has seen no visible key keeps m = -inf; pivot on 0 then
-      const float mc = m_used == -INFINITY ? 0.f : m_used * c;
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[BN / 2];
-#pragma unroll
-      for (int i = 0; i < BN / 2; ++i) {
-        const float p0 = ex2(fmaf(s[2 * i], c, -mc));
-        const float p1 = ex2(fmaf(s[2 * i + 1], c, -mc));
-        sum4[i % 4] += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
-      }
-      l = l * alpha + ((sum4[0] + sum4[1]) + (sum4[2] + sum4[3]));
+      // O picks up the new maximum before this tile's P V is accumulated into it
       if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
@@ -308,16 +317,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           tmem_st32(tO + cc * 32, r);
         }
       }
+      // a row that has seen no visible key keeps m = -inf; pivot on 0 then
+      const float mc = m_used == -INFINITY ? 0.f : m_used * c;
+      const uint64_t c2 = f2_pack(c, c), nmc2 = f2_pack(-mc, -mc);
+      uint64_t sum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+      // Exponentials in two halves of 64 keys; each half goes to tensor memory and
+      // is published at once so the P V MMA can start on it.
 #pragma unroll
-      for (int cc = 0; cc < BN / 64; ++cc) {
-        uint32_t r[32];
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) r[i] = pk[cc * 32 + i];
-        tmem_st32(tS + cc * 32, r);
+        for (int i = 0; i < 32; ++i) {
+          const int e = half * 64 + 2 * i;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), c2, nmc2), x0, x1);
+          const float p0 = ex2(x0), p1 = ex2(x1);
+          sum2[i % 2] = f2_add(sum2[i % 2], f2_pack(p0, p1));
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tS + half * 32, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(half ? &bars->p_hi[t] : &bars->p_lo[t]);
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars->p_full[t]);
+      float s0, s1, s2, s3;
+      f2_unpack(sum2[0], s0, s1);
+      f2_unpack(sum2[1], s2, s3);
+      l = l * alpha + ((s0 + s1) + (s2 + s3));
     }
     if (ok && n > 0) ok = mbar_wait(&bars->o_full, 0, 20 + t);
     if (ok && n > 0) {
