@@ -79,6 +79,22 @@ bool make_map(CUtensorMap* map, const void* base, int d, int N, int BH) {
   return r == CUDA_SUCCESS;
 }
 
+// 3-D fp32 view {d, N, B*H} of the backward pass's dQ accumulator, box
+// {32, 32, 1} (128-byte rows), 128-byte swizzle: the target of the bulk
+// reduce-adds.
+bool make_dq_map(CUtensorMap* map, void* acc, int d, int N, int BH) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 4, (cuuint64_t)N * d * 4};
+  const cuuint32_t box[3] = {32, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, acc, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // The tcgen05 kernels need an sm_100 device (compute capability 10.0).
 fa_status check_device() {
   int dev = 0;
@@ -150,12 +166,13 @@ fa_status fa_backward(const void* q, const void* k, const void* v, const void* o
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
   if ((s = check_device()) != FA_OK) return s;
   const int BH = B * H;
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   if (!make_map(&mq, q, d, N, BH) || !make_map(&mk, k, d, N, BH) || !make_map(&mv, v, d, N, BH) ||
-      !make_map(&mdo, dout, d, N, BH))
+      !make_map(&mdo, dout, d, N, BH) ||
+      !make_dq_map(&mdq, static_cast<char*>(workspace) + sm100_backward_dq_offset(BH, N), d, N, BH))
     return map_failed();
-  return from_cuda(sm100_backward(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, workspace, BH, N, d,
-                                  scale, causal ? 1 : 0, static_cast<cudaStream_t>(stream)));
+  return from_cuda(sm100_backward(mq, mk, mv, mdo, mdq, o, dout, lse, dq, dk, dv, workspace, BH, N,
+                                  d, scale, causal ? 1 : 0, static_cast<cudaStream_t>(stream)));
 }
 
 fa_status fa_backward_fp32(const float* q, const float* k, const float* v, const float* o,
@@ -245,10 +262,11 @@ extern "C" fa_status fa_backward_noalloc(const void* q, const void* k, const voi
   void* scratch = noalloc_scratch();
   if (scratch == nullptr) return FA_ERR_CUDA;
   const int BH = B * H;
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   if (!make_map(&mq, q, d, N, BH) || !make_map(&mk, k, d, N, BH) || !make_map(&mv, v, d, N, BH) ||
-      !make_map(&mdo, dout, d, N, BH))
+      !make_map(&mdo, dout, d, N, BH) ||
+      !make_dq_map(&mdq, static_cast<char*>(scratch) + sm100_backward_dq_offset(BH, N), d, N, BH))
     return map_failed();
-  return from_cuda(sm100_backward(mq, mk, mv, mdo, o, dout, lse, dq, dk, dv, scratch, BH, N, d,
+  return from_cuda(sm100_backward(mq, mk, mv, mdo, mdq, o, dout, lse, dq, dk, dv, scratch, BH, N, d,
                                   scale, causal ? 1 : 0, static_cast<cudaStream_t>(stream)));
 }

@@ -15,14 +15,15 @@
 //               forms P^T (to tensor memory) and dS (to shared memory), then
 //               accumulates dV += P^T dO and dK += dS^T Q in tensor memory and
 //               computes the partial dQ = dS K, which a reduce group adds into
-//               the fp32 accumulator with vector atomics;
+//               the fp32 accumulator with bulk tensor reduce-adds;
 //   convert     dQ = scale * accumulator, rounded to bf16.
 //
 // Main-kernel CTA layout (512 threads, registers rebalanced with setmaxnreg):
 //   warps 0-7   P / dS computation (thread = key row = tensor-memory lane, two
 //               warps per row quarter, one per half of the query columns) and
 //               the dK / dV epilogue
-//   warps 8-11  dQ drain: tensor memory -> registers -> red.global.add.v2.f32
+//   warps 8-11  dQ drain: tensor memory -> registers -> shared staging -> bulk
+//               tensor reduce-add into the fp32 accumulator
 //   warp  12    TMA producer: K, V once; Q_i, dO_i, LSE_i, D_i per query tile
 //   warp  13    tensor-memory allocator and MMA issuer (warps 14-15 idle)
 // Tensor memory: S^T at column 0 (P^T of query columns 64h.. packed at column 64h),
@@ -48,11 +49,11 @@ constexpr int NTHREADS = 512;     // four warpgroups
 constexpr int kProducerWarp = 12;
 constexpr int kMmaWarp = 13;
 // Register split (setmaxnreg).  The launch gives every thread 128 registers,
-// 512 * 128 = 65536 in all; the shares below sum to 128 * (2*144 + 136 + 88) =
+// 512 * 128 = 65536 in all; the shares below sum to 128 * (2*136 + 160 + 80) =
 // 65536, exactly that pool.
-constexpr int kRegsCompute = 144;  // warpgroups 0 and 1
-constexpr int kRegsReduce = 136;   // warpgroup 2
-constexpr int kRegsControl = 88;   // warpgroup 3: producer, MMA issuer, two idle warps
+constexpr int kRegsCompute = 136;  // warpgroups 0 and 1
+constexpr int kRegsReduce = 160;   // warpgroup 2
+constexpr int kRegsControl = 80;   // warpgroup 3: producer, MMA issuer, two idle warps
 static_assert(128 * (2 * kRegsCompute + kRegsReduce + kRegsControl) <= 512 * 128,
               "register split exceeds the launch allocation");
 constexpr int NST = 2;  // Q / dO stages
@@ -64,9 +65,12 @@ struct Cfg {
   static constexpr int CHUNK = BN * 128;   // one 64-column swizzle chunk of a tile
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = TILE;
-  static constexpr int OFF_STAGE = 2 * TILE;       // stage s: Q at +0, dO at +TILE
-  static constexpr int OFF_DS = OFF_STAGE + NST * 2 * TILE;
-  static constexpr int OFF_VEC = OFF_DS + BM * BN * 2;  // LSE2 / D vectors per stage
+  static constexpr int OFF_Q = 2 * TILE;                   // stage s at OFF_Q + s * TILE
+  static constexpr int OFF_DO = OFF_Q + NST * TILE;        // dO: one buffer
+  static constexpr int OFF_DS = OFF_DO + TILE;
+  static constexpr int OFF_STG = OFF_DS + BM * BN * 2;     // dQ staging: 4 warps x 2 x 4 KB
+  static constexpr int STG_BYTES = 32 * 32 * 4;            // 32 rows x 32 fp32 columns
+  static constexpr int OFF_VEC = OFF_STG + 4 * 2 * STG_BYTES;  // LSE2 / D vectors per stage
   static constexpr int OFF_BAR = OFF_VEC + NST * 2 * BM * 4;
   static constexpr int SMEM_BYTES = OFF_BAR + 256;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -93,8 +97,10 @@ struct Params {
 
 struct Bars {
   uint64_t kv_full;
-  uint64_t qdo_full[NST];
-  uint64_t qdo_empty[NST];
+  uint64_t q_full[NST];    // Q tile + LSE2 / D vectors of a stage
+  uint64_t q_empty[NST];
+  uint64_t do_full;        // dO tile (single buffer)
+  uint64_t do_empty;
   uint64_t s_full;
   uint64_t dp_full;
   uint64_t p_full;
@@ -107,14 +113,15 @@ struct Bars {
   uint32_t tmem_base;
 };
 
-__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
-}
 
-__device__ __forceinline__ void red_add_v2(float* addr, float a, float b) {
-  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(addr), "f"(a), "f"(b) : "memory");
+// Bulk tensor reduce-add of a shared-memory box into global memory (async proxy).
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, uint32_t src_smem, int c0,
+                                                  int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src_smem), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
 }
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -147,7 +154,7 @@ template <int D>
 __global__ void __launch_bounds__(NTHREADS, 1)
     main_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                 const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
-                const Params p) {
+                const __grid_constant__ CUtensorMap mdq, const Params p) {
   using C = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   // The swizzled tiles need a 1024-byte aligned base and the layout uses the
@@ -175,9 +182,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < NST; ++s) {
-      mbar_init(&bars->qdo_full[s], 1);
-      mbar_init(&bars->qdo_empty[s], 1);
+      mbar_init(&bars->q_full[s], 1);
+      mbar_init(&bars->q_empty[s], 1);
     }
+    mbar_init(&bars->do_full, 1);
+    mbar_init(&bars->do_empty, 1);
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
     mbar_init(&bars->p_full, 2 * 128);
@@ -198,6 +207,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tma_prefetch_desc(&mk);
     tma_prefetch_desc(&mv);
     tma_prefetch_desc(&mdo);
+    tma_prefetch_desc(&mdq);
   }
   tc_fence_before();
   __syncthreads();
@@ -214,43 +224,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tma_load_3d(sV + c * C::CHUNK, &mv, &bars->kv_full, c * 64, j * BN, bh);
       }
       bool ok = true;
-      int issued = 0;
+      int issued = 0, do_issued = 0;
       for (int it = 0; it < niter && ok; ++it) {
         const int st = it % NST, round = it / NST;
-        if (round > 0) ok = mbar_wait(&bars->qdo_empty[st], (round - 1) & 1, 32);
-        if (!ok) break;
         const int i = i0 + it;
-        uint8_t* sQ = smem + C::OFF_STAGE + st * 2 * C::TILE;
-        uint8_t* sdO = sQ + C::TILE;
+        if (round > 0) ok = mbar_wait(&bars->q_empty[st], (round - 1) & 1, 32);
+        if (!ok) break;
+        uint8_t* sQ = smem + C::OFF_Q + st * C::TILE;
         float* vec = sVec + st * 2 * BM;
-        mbar_arrive_expect_tx(&bars->qdo_full[st], 2 * C::TILE + 2 * BM * 4);
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(sQ + c * C::CHUNK, &mq, &bars->qdo_full[st], c * 64, i * BM, bh);
-          tma_load_3d(sdO + c * C::CHUNK, &mdo, &bars->qdo_full[st], c * 64, i * BM, bh);
-        }
+        mbar_arrive_expect_tx(&bars->q_full[st], C::TILE + 2 * BM * 4);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sQ + c * C::CHUNK, &mq, &bars->q_full[st], c * 64, i * BM, bh);
         const size_t voff = (size_t)bh * p.Npad + (size_t)i * BM;
-        bulk_load(vec, p.lse2 + voff, BM * 4, &bars->qdo_full[st]);
-        bulk_load(vec + BM, p.dsum + voff, BM * 4, &bars->qdo_full[st]);
+        bulk_load(vec, p.lse2 + voff, BM * 4, &bars->q_full[st]);
+        bulk_load(vec + BM, p.dsum + voff, BM * 4, &bars->q_full[st]);
         issued = it + 1;
+        // dO of tile i reuses the single dO buffer once dV of tile i-1 has read it
+        if (it > 0) ok = mbar_wait(&bars->do_empty, (it - 1) & 1, 47);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bars->do_full, C::TILE);
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + C::OFF_DO + c * C::CHUNK, &mdo, &bars->do_full, c * 64, i * BM, bh);
+        do_issued = it + 1;
       }
       mbar_wait(&bars->kv_full, 0, 33);
       for (int s = 0; s < NST && s < issued; ++s) {
         const int last = s + ((issued - 1 - s) / NST) * NST;
-        mbar_wait(&bars->qdo_full[s], (last / NST) & 1, 34);
+        mbar_wait(&bars->q_full[s], (last / NST) & 1, 34);
       }
+      if (do_issued > 0) mbar_wait(&bars->do_full, (do_issued - 1) & 1, 48);
     }
    } else if (warp == kMmaWarp) {
     if (lane == 0) {
       const uint32_t uK = smem_u32(sK), uV = smem_u32(sV), uDS = smem_u32(sDS);
-      bool ok = mbar_wait(&bars->kv_full, 0, 35);
-      for (int it = 0; it < niter && ok; ++it) {
-        const int st = it % NST;
-        const uint32_t uQ = smem_u32(smem + C::OFF_STAGE + st * 2 * C::TILE);
-        const uint32_t udO = uQ + C::TILE;
-        ok = mbar_wait(&bars->qdo_full[st], (it / NST) & 1, 36);
-        if (!ok) break;
-        tc_fence_after();
-        // S^T = K Q^T  (keys x queries), K = d
+      auto stage_q = [&](int it) { return smem_u32(smem + C::OFF_Q + (it % NST) * C::TILE); };
+      const uint32_t udO = smem_u32(smem + C::OFF_DO);
+      // S^T = K Q^T  (keys x queries), K = d
+      auto issue_s = [&](int it) {
+        const uint32_t uQ = stage_q(it);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
@@ -258,12 +269,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  C::IDESC_S, kk > 0);
         }
         mma_commit(&bars->s_full);
-        if (it > 0) {
-          ok = mbar_wait(&bars->dq_empty, (it - 1) & 1, 37);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        // dP^T = V dO^T
+      };
+      // dP^T = V dO^T
+      auto issue_dp = [&](int it) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
@@ -271,19 +279,51 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  C::IDESC_S, kk > 0);
         }
         mma_commit(&bars->dp_full);
-        ok = mbar_wait(&bars->p_full, it & 1, 46);
-        if (!ok) break;
-        tc_fence_after();
-        // dV += P^T dO  (keys x d), K = 128 queries, P^T from tensor memory (queries
-        // 64h .. 64h+63 packed at column 64h); runs while the compute warps form dS
+      };
+      // dV += P^T dO  (keys x d), K = 128 queries, P^T from tensor memory (queries
+      // 64h .. 64h+63 packed at column 64h)
+      auto issue_dv = [&](int it) {
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
           mma_ts(tmem + C::T_DV, tmem + C::T_S + 64 * (kk / 4) + 8 * (kk % 4),
-                 sdesc_sw128(udO + kk * 2048, C::CHUNK, 1024),
-                 C::IDESC_DKV, (it > 0 || kk > 0) ? 1u : 0u);
+                 sdesc_sw128(udO + kk * 2048, C::CHUNK, 1024), C::IDESC_DKV,
+                 (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&bars->do_empty);
+      };
+      // Order per query tile i (after the prologue S(0), dP(0), dV(0)):
+      //   S(i+1) | dQ(i) | dK(i) | dP(i+1) | dV(i+1)
+      // S(i+1) goes ahead of dQ(i) and dK(i) (dV(i) has already read P^T(i) from the
+      // S columns), so the compute warps form P(i+1) while the tensor core runs
+      // dQ(i) and dK(i).
+      bool ok = mbar_wait(&bars->kv_full, 0, 35);
+      if (ok) ok = mbar_wait(&bars->q_full[0], 0, 36);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        ok = mbar_wait(&bars->do_full, 0, 49);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_dp(0);
+        ok = mbar_wait(&bars->p_full, 0, 46);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_dv(0);
+      }
+      for (int it = 0; it < niter && ok; ++it) {
+        const int st = it % NST;
+        const uint32_t uQ = stage_q(it);
         ok = mbar_wait(&bars->ds_full, it & 1, 38);
         if (!ok) break;
         tc_fence_after();
+        const bool more = it + 1 < niter;
+        if (more) {
+          ok = mbar_wait(&bars->q_full[(it + 1) % NST], ((it + 1) / NST) & 1, 36);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(it + 1);
+        }
         // dQ_part = dS K  (queries x d), K = 128 keys; written over dP^T
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
@@ -299,7 +339,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  (it > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&bars->ds_free);
-        mma_commit(&bars->qdo_empty[st]);
+        mma_commit(&bars->q_empty[st]);
+        if (more) {
+          ok = mbar_wait(&bars->dq_empty, it & 1, 37);
+          if (ok) ok = mbar_wait(&bars->do_full, (it + 1) & 1, 49);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dp(it + 1);
+          ok = mbar_wait(&bars->p_full, (it + 1) & 1, 46);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dv(it + 1);
+        }
       }
       if (ok) mma_commit(&bars->all_done);
       mma_commit(&bars->drain);
@@ -309,12 +360,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsCompute));
     // Compute warps 0-7.  Warp w owns tensor-memory lane quarter w % 4 (key rows
-    // 32*(w%4) .. +31 for S^T/dP^T/dK/dV, query rows for dQ) and column half
-    // h = w / 4: query columns 64h .. 64h+63 of P^T and dS, dQ / dK / dV columns
-    // (d/2)h .. (d/2)h + d/2 - 1.  Per query tile: P^T -> tensor memory, dS ->
-    // shared memory, then the partial dQ of the tile is drained from tensor memory
-    // and added to the fp32 accumulator while the tensor core runs dK and the next
-    // tile's S^T and dP^T.
+    // 32*(w%4) .. +31 for S^T/dP^T/dK/dV) and column half h = w / 4: query
+    // columns 64h .. 64h+63 of P^T and dS, dK / dV columns (d/2)h .. +d/2-1.  Per
+    // query tile: P^T -> tensor memory, dS -> shared memory.
     const int qw = warp % 4, h = warp / 4;
     const int r = qw * 32 + lane;
     const int kr = j * BN + r;
@@ -330,7 +378,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int i = i0 + it, st = it % NST;
       const uint32_t lse2 = smem_u32(sVec + st * 2 * BM) + h * 64 * 4;  // LSE*log2(e), my columns
       const uint32_t dsv = lse2 + BM * 4;                                // D, my columns
-      ok = mbar_wait(&bars->qdo_full[st], (it / NST) & 1, 40);
+      ok = mbar_wait(&bars->q_full[st], (it / NST) & 1, 40);
       if (ok) ok = mbar_wait(&bars->s_full, it & 1, 41);
       if (!ok) break;
       tc_fence_after();
@@ -426,41 +474,49 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsReduce));
     // dQ reduce warps 8-11: warp w drains query rows 32*(w%4) .. +31 of each
-    // tile's partial dQ from tensor memory and adds them to the fp32 accumulator.
-    // It reads 16 rows x 64 columns at a time in the 16x256b shape, where four
-    // adjacent lanes hold 8 contiguous columns of one row, so each
-    // red.global.add.v2 instruction covers 8 rows x 32 contiguous bytes.
+    // tile's partial dQ from tensor memory, then, 32 columns at a time, writes
+    // them to its own 128-byte-swizzled 4 KB staging buffer (two per warp, used
+    // in turn) and lane 0 adds the buffer into the fp32 accumulator with one
+    // bulk tensor reduce-add.  No per-thread global atomics.
     const int qw = warp % 4;
     const uint32_t tQ = tmem + ((uint32_t)(qw * 32) << 16) + C::T_DP;
+    const uint32_t stg0 = smem_u32(smem + C::OFF_STG + qw * 2 * C::STG_BYTES);
     bool ok = true;
+    int chunk = 0;
     for (int it = 0; it < niter && ok; ++it) {
       ok = mbar_wait(&bars->dq_full, it & 1, 45);
       if (!ok) break;
       tc_fence_after();
-      const int tile_row = (i0 + it) * BM + qw * 32 + lane / 4;
-      constexpr int NPART = 2 * (D / 64);
+      uint32_t v[D / 32][32];
 #pragma unroll
-      for (int part = 0; part < NPART; ++part) {
-        const int hh = part / (D / 64), ch = part % (D / 64);  // lane half, 64-column block
-        uint32_t v[32];
-        tmem_ld16x256b_x8(tQ + ((uint32_t)(16 * hh) << 16) + ch * 64, v);
-        tmem_wait_ld();
-        if (part == NPART - 1) {
-          tc_fence_before();
-          mbar_arrive(&bars->dq_empty);
+      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tQ + cc * 32, v[cc]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars->dq_empty);
+      const int row0 = (i0 + it) * BM + qw * 32;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc, ++chunk) {
+        const uint32_t buf = stg0 + (chunk & 1) * C::STG_BYTES;
+        if (chunk >= 2) {
+          // the reduce that read this buffer two chunks ago must be done with it
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+          __syncwarp();
         }
-        const int r0 = tile_row + 16 * hh, r1 = r0 + 8;
-        const int col = ch * 64 + 2 * (lane % 4);
-        float* d0 = p.dq_acc + ((size_t)bh * p.N + r0) * D + col;
-        float* d1 = p.dq_acc + ((size_t)bh * p.N + r1) * D + col;
 #pragma unroll
-        for (int jb = 0; jb < 8; ++jb) {
-          if (r0 < p.N) red_add_v2(d0 + 8 * jb, __uint_as_float(v[4 * jb]), __uint_as_float(v[4 * jb + 1]));
-          if (r1 < p.N)
-            red_add_v2(d1 + 8 * jb, __uint_as_float(v[4 * jb + 2]), __uint_as_float(v[4 * jb + 3]));
+        for (int u = 0; u < 8; ++u)
+          st_shared_v4(buf + lane * 128 + ((u ^ (lane & 7)) << 4), v[cc][4 * u], v[cc][4 * u + 1],
+                       v[cc][4 * u + 2], v[cc][4 * u + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          // rows past N are clipped by the tensor map; a box wholly past N is skipped
+          if (row0 < p.N) tma_reduce_add_3d(&mdq, buf, cc * 32, row0, bh);
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
         }
       }
     }
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -532,8 +588,14 @@ size_t sm100_backward_workspace(int BH, int N, int d) {
   return 2 * vec + acc;
 }
 
+size_t sm100_backward_dq_offset(int BH, int N) {
+  const size_t npad = (size_t)(N + 127) / 128 * 128;
+  return 2 * (((size_t)BH * npad * 4 + 255) / 256 * 256);
+}
+
 cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                           const CUtensorMap& mdo, const void* o, const void* dout, const float* lse,
+                           const CUtensorMap& mdo, const CUtensorMap& mdq, const void* o,
+                           const void* dout, const float* lse,
                            void* dq, void* dk, void* dv, void* workspace, int BH, int N, int d,
                            float scale, int causal, cudaStream_t st) {
   const int npad = (N + 127) / 128 * 128;
@@ -570,12 +632,12 @@ cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const C
     const int smem = bwd::Cfg<128>::SMEM_BYTES;
     e = cudaFuncSetAttribute(bwd::main_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    bwd::main_kernel<128><<<grid, bwd::NTHREADS, smem, st>>>(mq, mk, mv, mdo, p);
+    bwd::main_kernel<128><<<grid, bwd::NTHREADS, smem, st>>>(mq, mk, mv, mdo, mdq, p);
   } else {
     const int smem = bwd::Cfg<64>::SMEM_BYTES;
     e = cudaFuncSetAttribute(bwd::main_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    bwd::main_kernel<64><<<grid, bwd::NTHREADS, smem, st>>>(mq, mk, mv, mdo, p);
+    bwd::main_kernel<64><<<grid, bwd::NTHREADS, smem, st>>>(mq, mk, mv, mdo, mdq, p);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;

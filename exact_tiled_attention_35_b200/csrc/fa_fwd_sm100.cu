@@ -35,6 +35,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "fa_device.cuh"
 #include "fa_kernels.h"
 
@@ -76,6 +78,7 @@ struct Params {
   int BH;
   int N;
   int npairs;  // ceil(N / 256)
+  int group;   // heads per scheduling group (their K/V stay resident in L2)
   float scale;
   float scale_log2;
   int causal;
@@ -114,10 +117,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // heavy tiles first under the causal mask: pair index runs backwards
+  // Blocks run in groups of p.group heads so that the K/V those CTAs share stay
+  // in L2; inside a group, heavy tiles come first under the causal mask (the
+  // pair index runs backwards).
   const int blk = blockIdx.x;
-  const int bh = blk % p.BH;
-  const int pair = p.causal ? (p.npairs - 1 - blk / p.BH) : (blk / p.BH);
+  const int full_blocks = (p.BH / p.group) * p.group * p.npairs;
+  int bh, rank;
+  if (blk < full_blocks) {
+    const int g = blk / (p.group * p.npairs), r = blk % (p.group * p.npairs);
+    bh = g * p.group + r % p.group;
+    rank = r / p.group;
+  } else {
+    const int gt = p.BH % p.group, r = blk - full_blocks;
+    bh = (p.BH / p.group) * p.group + r % gt;
+    rank = r / gt;
+  }
+  const int pair = p.causal ? (p.npairs - 1 - rank) : rank;
   const int qbase = pair * (NQT * BM);
   int ntile[NQT];
 #pragma unroll
@@ -389,6 +404,9 @@ cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   p.BH = BH;
   p.N = N;
   p.npairs = (N + 2 * fwd::BM - 1) / (2 * fwd::BM);
+  // heads whose K and V (4 N d bytes each) fit in about 48 MB of the 126 MB L2
+  const long long kv_bytes = 4LL * N * d;
+  p.group = (int)std::max(1LL, std::min<long long>(BH, (48LL << 20) / kv_bytes));
   p.scale = scale;
   p.scale_log2 = scale * fwd::kLog2e;
   p.causal = causal;

@@ -24,8 +24,12 @@ cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CU
 // tcgen05 backward (fa_bwd_sm100.cu): preprocess, main and dQ-convert kernels.
 // Workspace layout: LSE*log2(e) [BH, Npad], D [BH, Npad], fp32 dQ [BH, N, d].
 size_t sm100_backward_workspace(int BH, int N, int d);
+// byte offset of the fp32 dQ accumulator inside the workspace
+size_t sm100_backward_dq_offset(int BH, int N);
+// mdq: 3-D fp32 view {d, N, B*H} of the accumulator, box {32, 32, 1}, 128-byte swizzle
 cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                           const CUtensorMap& mdo, const void* o, const void* dout, const float* lse,
+                           const CUtensorMap& mdo, const CUtensorMap& mdq, const void* o,
+                           const void* dout, const float* lse,
                            void* dq, void* dk, void* dv, void* workspace, int BH, int N, int d,
                            float scale, int causal, cudaStream_t st);
 
