@@ -7,9 +7,9 @@
 //   D_i = sum_c dO[i,c] O[i,c],  dQ = scale * dS K,  dK = scale * dS^T Q.
 //
 // Three kernels:
-//   preprocess  D, LSE * log2(e) (padded to whole 128-row tiles: padding rows get
-//               LSE = +inf so their probabilities vanish) and a zeroed fp32 dQ
-//               accumulator;
+//   preprocess  -D and -LSE * log2(e) (padded to whole 128-row tiles: padding
+//               rows get +inf for LSE so their probabilities vanish) and a zeroed
+//               fp32 dQ accumulator;
 //   main        one CTA per 128-key tile; for every 128-row query tile it
 //               recomputes S^T = K Q^T and dP^T = V dO^T in tensor memory,
 //               forms P^T (to tensor memory) and dS (to shared memory), then
@@ -49,11 +49,11 @@ constexpr int NTHREADS = 512;     // four warpgroups
 constexpr int kProducerWarp = 12;
 constexpr int kMmaWarp = 13;
 // Register split (setmaxnreg).  The launch gives every thread 128 registers,
-// 512 * 128 = 65536 in all; the shares below sum to 128 * (2*136 + 160 + 80) =
+// 512 * 128 = 65536 in all; the shares below sum to 128 * (2*136 + 144 + 96) =
 // 65536, exactly that pool.
 constexpr int kRegsCompute = 136;  // warpgroups 0 and 1
-constexpr int kRegsReduce = 160;   // warpgroup 2
-constexpr int kRegsControl = 80;   // warpgroup 3: producer, MMA issuer, two idle warps
+constexpr int kRegsReduce = 144;   // warpgroup 2
+constexpr int kRegsControl = 96;   // warpgroup 3: producer, MMA issuer, two idle warps
 static_assert(128 * (2 * kRegsCompute + kRegsReduce + kRegsControl) <= 512 * 128,
               "register split exceeds the launch allocation");
 constexpr int NST = 2;  // Q / dO stages
@@ -84,8 +84,8 @@ struct Params {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   float* dq_acc;       // [BH, N, d] fp32
-  const float* lse2;   // [BH, Npad]  LSE * log2(e), +inf on padding rows
-  const float* dsum;   // [BH, Npad]  D, 0 on padding rows
+  const float* lse2;   // [BH, Npad]  -LSE * log2(e), -inf on padding rows
+  const float* dsum;   // [BH, Npad]  -D, 0 on padding rows
   int BH;
   int N;
   int Npad;
@@ -290,11 +290,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                  (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->do_empty);
       };
-      // Order per query tile i (after the prologue S(0), dP(0), dV(0)):
-      //   S(i+1) | dQ(i) | dK(i) | dP(i+1) | dV(i+1)
-      // S(i+1) goes ahead of dQ(i) and dK(i) (dV(i) has already read P^T(i) from the
-      // S columns), so the compute warps form P(i+1) while the tensor core runs
-      // dQ(i) and dK(i).
+      // Order per query tile i (after the prologue S(0), dP(0)):
+      //   dV(i) | S(i+1) | dQ(i) | dK(i) | dP(i+1)
+      // S(i+1) is issued as soon as dV(i) has read P^T(i) from the S columns (the
+      // compute warps no longer touch them in tile i), so it runs while they form
+      // dS(i); dQ(i) and dK(i) then run while they form P(i+1).
       bool ok = mbar_wait(&bars->kv_full, 0, 35);
       if (ok) ok = mbar_wait(&bars->q_full[0], 0, 36);
       if (ok) {
@@ -305,25 +305,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       if (ok) {
         tc_fence_after();
         issue_dp(0);
-        ok = mbar_wait(&bars->p_full, 0, 46);
-      }
-      if (ok) {
-        tc_fence_after();
-        issue_dv(0);
       }
       for (int it = 0; it < niter && ok; ++it) {
         const int st = it % NST;
         const uint32_t uQ = stage_q(it);
-        ok = mbar_wait(&bars->ds_full, it & 1, 38);
+        const bool more = it + 1 < niter;
+        ok = mbar_wait(&bars->p_full, it & 1, 46);
         if (!ok) break;
         tc_fence_after();
-        const bool more = it + 1 < niter;
+        issue_dv(it);
         if (more) {
           ok = mbar_wait(&bars->q_full[(it + 1) % NST], ((it + 1) / NST) & 1, 36);
           if (!ok) break;
           tc_fence_after();
           issue_s(it + 1);
         }
+        ok = mbar_wait(&bars->ds_full, it & 1, 38);
+        if (!ok) break;
+        tc_fence_after();
         // dQ_part = dS K  (queries x d), K = 128 keys; written over dP^T
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
@@ -346,10 +345,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (!ok) break;
           tc_fence_after();
           issue_dp(it + 1);
-          ok = mbar_wait(&bars->p_full, (it + 1) & 1, 46);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dv(it + 1);
         }
       }
       if (ok) mma_commit(&bars->all_done);
@@ -376,8 +371,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     bool ok = true;
     for (int it = 0; it < niter && ok; ++it) {
       const int i = i0 + it, st = it % NST;
-      const uint32_t lse2 = smem_u32(sVec + st * 2 * BM) + h * 64 * 4;  // LSE*log2(e), my columns
-      const uint32_t dsv = lse2 + BM * 4;                                // D, my columns
+      const uint32_t lse2 = smem_u32(sVec + st * 2 * BM) + h * 64 * 4;  // -LSE*log2(e), my columns
+      const uint32_t dsv = lse2 + BM * 4;                                // -D, my columns
       ok = mbar_wait(&bars->q_full[st], (it / NST) & 1, 40);
       if (ok) ok = mbar_wait(&bars->s_full, it & 1, 41);
       if (!ok) break;
@@ -392,17 +387,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tmem_wait_ld();
       const bool diag = p.causal && i == j;
+      const uint64_t c2 = f2_pack(c, c);
 #pragma unroll
       for (int c4 = 0; c4 < 16; ++c4) {
         const float4 l4 = ld_shared_v4(lse2 + c4 * 16);
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+        // x = s * c - LSE * log2(e) for two columns at a time (the vector holds -LSE * log2(e))
+        float x0, x1, x2, x3;
+        f2_unpack(f2_fma(f2_pack(pr[4 * c4], pr[4 * c4 + 1]), c2, f2_pack(l4.x, l4.y)), x0, x1);
+        f2_unpack(f2_fma(f2_pack(pr[4 * c4 + 2], pr[4 * c4 + 3]), c2, f2_pack(l4.z, l4.w)), x2, x3);
+        pr[4 * c4] = ex2(x0);
+        pr[4 * c4 + 1] = ex2(x1);
+        pr[4 * c4 + 2] = ex2(x2);
+        pr[4 * c4 + 3] = ex2(x3);
+      }
+      if (!key_ok || diag) {  // masked keys: rows past N, and keys above the diagonal
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int col = c4 * 4 + e;
-          float pv = ex2(fmaf(pr[col], c, -lv[e]));
-          if (!key_ok || (diag && h * 64 + col < r)) pv = 0.f;
-          pr[col] = pv;
-        }
+        for (int col = 0; col < 64; ++col)
+          if (!key_ok || h * 64 + col < r) pr[col] = 0.f;
       }
       {
         uint32_t v[32];
@@ -428,10 +429,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int e4 = 0; e4 < 8; ++e4) {
           const int c0 = cc * 32 + 4 * e4;
           const float4 dd = ld_shared_v4(dsv + c0 * 4);
-          w[2 * e4] = pack_bf16x2(pr[c0] * (__uint_as_float(v[4 * e4]) - dd.x),
-                                  pr[c0 + 1] * (__uint_as_float(v[4 * e4 + 1]) - dd.y));
-          w[2 * e4 + 1] = pack_bf16x2(pr[c0 + 2] * (__uint_as_float(v[4 * e4 + 2]) - dd.z),
-                                      pr[c0 + 3] * (__uint_as_float(v[4 * e4 + 3]) - dd.w));
+          // dS = P * (dP - D), two columns per packed instruction (the vector holds -D)
+          float d0, d1, d2, d3;
+          f2_unpack(f2_mul(f2_pack(pr[c0], pr[c0 + 1]),
+                           f2_add(f2_pack(__uint_as_float(v[4 * e4]), __uint_as_float(v[4 * e4 + 1])),
+                                  f2_pack(dd.x, dd.y))), d0, d1);
+          f2_unpack(f2_mul(f2_pack(pr[c0 + 2], pr[c0 + 3]),
+                           f2_add(f2_pack(__uint_as_float(v[4 * e4 + 2]), __uint_as_float(v[4 * e4 + 3])),
+                                  f2_pack(dd.z, dd.w))), d2, d3);
+          w[2 * e4] = pack_bf16x2(d0, d1);
+          w[2 * e4 + 1] = pack_bf16x2(d2, d3);
         }
         // row r of the dS^T tile in the 128-byte swizzled layout: chunk h,
         // 16-byte units cc*4 .. cc*4+3 XOR (r % 8)
@@ -527,7 +534,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-// D, LSE*log2(e) (padded) and a zeroed dQ accumulator; one warp per padded row.
+// -D, -LSE*log2(e) (padded; the main kernel adds them) and a zeroed dQ
+// accumulator; one warp per padded row.
 template <int D>
 __global__ void __launch_bounds__(256) preprocess_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dout,
@@ -542,7 +550,7 @@ __global__ void __launch_bounds__(256) preprocess_kernel(const __nv_bfloat16* __
   const int bh = (int)(gw / Npad), row = (int)(gw % Npad);
   if (row >= N) {
     if (lane == 0) {
-      lse2[gw] = INFINITY;
+      lse2[gw] = -INFINITY;  // padding rows: probability exp2(-inf) = 0
       dsum[gw] = 0.f;
     }
     return;
@@ -561,8 +569,8 @@ __global__ void __launch_bounds__(256) preprocess_kernel(const __nv_bfloat16* __
   float4* z = reinterpret_cast<float4*>(dq_acc + off);
   for (int c = lane; c < D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (lane == 0) {
-    dsum[gw] = acc;
-    lse2[gw] = lse[(size_t)bh * N + row] * kLog2e;
+    dsum[gw] = -acc;
+    lse2[gw] = -lse[(size_t)bh * N + row] * kLog2e;
   }
 }
 
