@@ -17,7 +17,7 @@ import os
 
 import torch
 
-__all__ = ["forward", "backward", "backward_noalloc", "FAError", "library_path", "load_library", "check_device_status",
+__all__ = ["forward", "backward", "forward_gqa", "backward_gqa", "backward_noalloc", "FAError", "library_path", "load_library", "check_device_status",
            "workspace_size", "SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -27,9 +27,11 @@ _LIB = None
 _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SYMBOLS = {
     "fa_forward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_forward_gqa": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_forward_fp32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_workspace_size": (_Z, [_I, _I, _I, _I]),
     "fa_backward": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_backward_gqa": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_fp32": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_noalloc": (_I, [_P] * 9 + [_I, _I, _I, _I, _F, _I, _P]),
     "fa_check_device_status": (_I, [_P]),
@@ -127,6 +129,41 @@ def forward(q, k, v, causal=False, scale=None, out=None, lse=None):
     _check(fn(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d, scale, int(bool(causal)),
               _stream(q)), "fa_forward")
     return out, lse
+
+
+def forward_gqa(q, k, v, causal=False, scale=None, out=None, lse=None):
+    """Grouped-query / multi-query forward via fa_forward_gqa (bf16).
+
+    q: [B, H, N, d]; k, v: [B, Hkv, N, d] with Hkv dividing H."""
+    B, H, N, d = _shape(q)
+    Hkv = int(k.shape[1])
+    _require((q,), torch.bfloat16, (B, H, N, d))
+    _require((k, v), torch.bfloat16, (B, Hkv, N, d))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check(load_library().fa_forward_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, N,
+                                         d, scale, int(bool(causal)), _stream(q)), "fa_forward_gqa")
+    return out, lse
+
+
+def backward_gqa(q, k, v, o, do, lse, causal=False, scale=None, workspace=None):
+    """dQ [B,H,N,d], dK and dV [B,Hkv,N,d] via fa_backward_gqa (bf16)."""
+    B, H, N, d = _shape(q)
+    Hkv = int(k.shape[1])
+    _require((q, o, do), torch.bfloat16, (B, H, N, d))
+    _require((k, v), torch.bfloat16, (B, Hkv, N, d))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    lib = load_library()
+    if workspace is None:
+        workspace = torch.empty(max(int(lib.fa_backward_workspace_size(B, H, N, d)), 16),
+                                dtype=torch.uint8, device=q.device)
+    _check(lib.fa_backward_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                               _ptr(dk), _ptr(dv), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), B, H, Hkv, N, d, scale,
+                               int(bool(causal)), _stream(q)), "fa_backward_gqa")
+    return dq, dk, dv
 
 
 def workspace_size(B, H, N, d):

@@ -86,7 +86,10 @@ struct Params {
   float* dq_acc;       // [BH, N, d] fp32
   const float* lse2;   // [BH, Npad]  -LSE * log2(e), -inf on padding rows
   const float* dsum;   // [BH, Npad]  -D, 0 on padding rows
-  int BH;
+  int BH;      // query heads B*H
+  int BHkv;    // key/value heads B*Hkv
+  int H;       // query heads per batch
+  int G;       // query heads per key/value head (H / Hkv; 1 without grouping)
   int N;
   int Npad;
   int nkv;             // number of key tiles = Npad / 128
@@ -173,11 +176,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   // heavy key tiles first under the causal mask (tile j sees query tiles j..)
   const int blk = blockIdx.x;
-  const int bh = blk % p.BH;
-  const int j = blk / p.BH;
+  const int bkv = blk % p.BHkv;  // key/value head
+  const int j = blk / p.BHkv;
   const int nq = p.nkv;
   const int i0 = p.causal ? j : 0;
-  const int niter = nq - i0;
+  const int nqi = nq - i0;        // query tiles per query head
+  const int niter = p.G * nqi;    // every query head of the group, then its query tiles
+  // query head and query tile of iteration it
+  const int bhq0 = (bkv / (p.H / p.G)) * p.H + (bkv % (p.H / p.G)) * p.G;
+  auto q_head = [&](int it) { return bhq0 + it / nqi; };
+  auto q_tile = [&](int it) { return i0 + it % nqi; };
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -220,14 +228,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (lane == 0) {
       mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
       for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(sK + c * C::CHUNK, &mk, &bars->kv_full, c * 64, j * BN, bh);
-        tma_load_3d(sV + c * C::CHUNK, &mv, &bars->kv_full, c * 64, j * BN, bh);
+        tma_load_3d(sK + c * C::CHUNK, &mk, &bars->kv_full, c * 64, j * BN, bkv);
+        tma_load_3d(sV + c * C::CHUNK, &mv, &bars->kv_full, c * 64, j * BN, bkv);
       }
       bool ok = true;
       int issued = 0, do_issued = 0;
       for (int it = 0; it < niter && ok; ++it) {
         const int st = it % NST, round = it / NST;
-        const int i = i0 + it;
+        const int i = q_tile(it), bh = q_head(it);
         if (round > 0) ok = mbar_wait(&bars->q_empty[st], (round - 1) & 1, 32);
         if (!ok) break;
         uint8_t* sQ = smem + C::OFF_Q + st * C::TILE;
@@ -370,7 +378,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     constexpr int DH = D / 2;  // dQ / dK / dV columns per warp
     bool ok = true;
     for (int it = 0; it < niter && ok; ++it) {
-      const int i = i0 + it, st = it % NST;
+      const int i = q_tile(it), st = it % NST;
       const uint32_t lse2 = smem_u32(sVec + st * 2 * BM) + h * 64 * 4;  // -LSE*log2(e), my columns
       const uint32_t dsv = lse2 + BM * 4;                                // -D, my columns
       ok = mbar_wait(&bars->q_full[st], (it / NST) & 1, 40);
@@ -455,7 +463,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (ok) ok = mbar_wait(&bars->all_done, 0, 44);
     if (ok) {
       tc_fence_after();
-      const size_t row = (size_t)bh * p.N + (size_t)(key_ok ? kr : 0);
+      const size_t row = (size_t)bkv * p.N + (size_t)(key_ok ? kr : 0);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t tsrc = tmem + lane_off + (which ? C::T_DV : C::T_DK) + h * DH;
@@ -500,7 +508,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&bars->dq_empty);
-      const int row0 = (i0 + it) * BM + qw * 32;
+      const int row0 = q_tile(it) * BM + qw * 32, bh = q_head(it);
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc, ++chunk) {
         const uint32_t buf = stg0 + (chunk & 1) * C::STG_BYTES;
@@ -604,8 +612,9 @@ size_t sm100_backward_dq_offset(int BH, int N) {
 cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                            const CUtensorMap& mdo, const CUtensorMap& mdq, const void* o,
                            const void* dout, const float* lse,
-                           void* dq, void* dk, void* dv, void* workspace, int BH, int N, int d,
-                           float scale, int causal, cudaStream_t st) {
+                           void* dq, void* dk, void* dv, void* workspace, int B, int H, int Hkv,
+                           int N, int d, float scale, int causal, cudaStream_t st) {
+  const int BH = B * H;
   const int npad = (N + 127) / 128 * 128;
   const size_t vec = ((size_t)BH * npad * 4 + 255) / 256 * 256;
   float* lse2 = static_cast<float*>(workspace);
@@ -629,13 +638,16 @@ cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const C
   p.lse2 = lse2;
   p.dsum = dsum;
   p.BH = BH;
+  p.BHkv = B * Hkv;
+  p.H = H;
+  p.G = H / Hkv;
   p.N = N;
   p.Npad = npad;
   p.nkv = npad / 128;
   p.scale = scale;
   p.scale_log2 = scale * bwd::kLog2e;
   p.causal = causal;
-  const dim3 grid((unsigned)(p.nkv * BH));
+  const dim3 grid((unsigned)(p.nkv * p.BHkv));
   if (d == 128) {
     const int smem = bwd::Cfg<128>::SMEM_BYTES;
     e = cudaFuncSetAttribute(bwd::main_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

@@ -75,7 +75,9 @@ struct Cfg {
 struct Params {
   __nv_bfloat16* o;
   float* lse;
-  int BH;
+  int BH;      // query heads B*H
+  int H;       // query heads per batch
+  int G;       // query heads per key/value head (1 without grouping)
   int N;
   int npairs;  // ceil(N / 256)
   int group;   // heads per scheduling group (their K/V stay resident in L2)
@@ -133,6 +135,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     rank = r / gt;
   }
   const int pair = p.causal ? (p.npairs - 1 - rank) : rank;
+  // key/value head of query head bh (grouped-query attention; bh itself when G = 1)
+  const int bkv = (bh / p.H) * (p.H / p.G) + (bh % p.H) / p.G;
   const int qbase = pair * (NQT * BM);
   int ntile[NQT];
 #pragma unroll
@@ -192,7 +196,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         uint8_t* dst = sRing + slot * C::TILE;
         mbar_arrive_expect_tx(&bars->kv_full[slot], C::TILE);
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(dst + c * C::CHUNK, m, &bars->kv_full[slot], c * 64, j * BN, bh);
+          tma_load_3d(dst + c * C::CHUNK, m, &bars->kv_full[slot], c * 64, j * BN, bkv);
         issued = seq + 1;
       }
       // make sure no copy into this CTA's shared memory is still in flight at exit
@@ -396,12 +400,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }  // namespace fwd
 
 cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                          void* o, float* lse, int BH, int N, int d, float scale, int causal,
-                          cudaStream_t st) {
+                          void* o, float* lse, int B, int H, int Hkv, int N, int d, float scale,
+                          int causal, cudaStream_t st) {
+  const int BH = B * H;
   fwd::Params p;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.BH = BH;
+  p.H = H;
+  p.G = H / Hkv;
   p.N = N;
   p.npairs = (N + 2 * fwd::BM - 1) / (2 * fwd::BM);
   // heads whose K and V (4 N d bytes each) fit in about 48 MB of the 126 MB L2

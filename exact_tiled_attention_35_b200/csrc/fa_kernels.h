@@ -16,10 +16,11 @@ cudaError_t simt_backward(bool bf16, const void* q, const void* k, const void* v
                           int N, int d, float scale, int causal, cudaStream_t st);
 
 // tcgen05 forward (fa_fwd_sm100.cu).  Tensor maps: 3-D bf16 views
-// {d, N, B*H} of Q, K, V with a {64, 128, 1} box and 128-byte swizzle.
+// {d, N, heads} of Q (B*H heads), K and V (B*Hkv heads) with a {64, 128, 1} box
+// and 128-byte swizzle.  Hkv divides H (Hkv = H: plain multi-head attention).
 cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                          void* o, float* lse, int BH, int N, int d, float scale, int causal,
-                          cudaStream_t st);
+                          void* o, float* lse, int B, int H, int Hkv, int N, int d, float scale,
+                          int causal, cudaStream_t st);
 
 // tcgen05 backward (fa_bwd_sm100.cu): preprocess, main and dQ-convert kernels.
 // Workspace layout: LSE*log2(e) [BH, Npad], D [BH, Npad], fp32 dQ [BH, N, d].
@@ -30,7 +31,7 @@ size_t sm100_backward_dq_offset(int BH, int N);
 cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                            const CUtensorMap& mdo, const CUtensorMap& mdq, const void* o,
                            const void* dout, const float* lse,
-                           void* dq, void* dk, void* dv, void* workspace, int BH, int N, int d,
-                           float scale, int causal, cudaStream_t st);
+                           void* dq, void* dk, void* dv, void* workspace, int B, int H, int Hkv,
+                           int N, int d, float scale, int causal, cudaStream_t st);
 
 }  // namespace fa

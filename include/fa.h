@@ -60,13 +60,23 @@ typedef enum {
 fa_status fa_forward(const void* q, const void* k, const void* v, void* o, float* lse,
                      int B, int H, int N, int d, float scale, int causal, void* stream);
 
+/* Grouped-query / multi-query forward: K and V carry Hkv heads, [B,Hkv,N,d];
+ * query head h attends with key/value head h / (H / Hkv) (the attention
+ * variants named in "Atención Flash-2" of the unite.ai page).  Hkv must divide
+ * H; Hkv == H is fa_forward, Hkv == 1 is multi-query attention.  Q, O: [B,H,N,d];
+ * LSE: [B,H,N].  Errors as fa_forward, plus FA_ERR_INVALID_ARG for a bad Hkv. */
+fa_status fa_forward_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int B, int H, int Hkv, int N, int d, float scale, int causal,
+                         void* stream);
+
 /* Forward pass with fp32 storage (q, k, v, o are float [B,H,N,d]); fp32
  * arithmetic on CUDA cores.  Same definition, same LSE convention. */
 fa_status fa_forward_fp32(const float* q, const float* k, const float* v, float* o, float* lse,
                           int B, int H, int N, int d, float scale, int causal, void* stream);
 
-/* Bytes of device scratch fa_backward needs for this shape (0 on bad sizes).
- * It holds D_i = sum_c dO[i,c] * O[i,c] (fp32, [B,H,N]). */
+/* Bytes of device scratch fa_backward needs for this shape (0 on bad sizes):
+ * -LSE*log2(e) and -D_i = -sum_c dO[i,c] * O[i,c] padded to whole 128-row tiles
+ * (fp32, [B,H,Npad]) and an fp32 dQ accumulator ([B,H,N,d]). */
 size_t fa_backward_workspace_size(int B, int H, int N, int d);
 
 /* Backward pass, bf16 storage, fp32 accumulation.
@@ -81,6 +91,15 @@ fa_status fa_backward(const void* q, const void* k, const void* v, const void* o
                       const void* dout, const float* lse, void* dq, void* dk, void* dv,
                       void* workspace, size_t ws_bytes, int B, int H, int N, int d,
                       float scale, int causal, void* stream);
+
+/* Grouped-query / multi-query backward, the gradient of fa_forward_gqa:
+ * k, v, dk, dv are [B,Hkv,N,d]; dK and dV of a key/value head sum the
+ * contributions of its H / Hkv query heads.  q, o, dout, dq: [B,H,N,d].
+ * Workspace: fa_backward_workspace_size(B, H, N, d) (query heads). */
+fa_status fa_backward_gqa(const void* q, const void* k, const void* v, const void* o,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                          void* workspace, size_t ws_bytes, int B, int H, int Hkv, int N, int d,
+                          float scale, int causal, void* stream);
 
 /* Backward pass with fp32 storage (all tensors float); CUDA-core arithmetic.
  * Workspace as for fa_backward. */

@@ -5,7 +5,9 @@ and by the CPU-baseline leg of ``bench.py``; never by the library.
 """
 
 from .attention import (  # noqa: F401
+    attention_bwd_gqa_ref,
     attention_bwd_ref,
+    attention_fwd_gqa_ref,
     attention_fwd_ref,
     attention_rows_ref,
     online_softmax_attention,

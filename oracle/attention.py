@@ -45,6 +45,8 @@ __all__ = [
     "attention_bwd_ref",
     "attention_rows_ref",
     "online_softmax_attention",
+    "attention_fwd_gqa_ref",
+    "attention_bwd_gqa_ref",
 ]
 
 
@@ -221,3 +223,34 @@ def online_softmax_attention(q, k, v, scale, causal, block_q=128, block_k=128):
                 o[b, h, i0:i1] = ob
                 lse[b, h, i0:i1] = (mrow + np.log(lrow))[:, 0]
     return o, lse
+
+
+def _repeat_heads(x, group):
+    """[B, Hkv, N, d] -> [B, Hkv*group, N, d]: key/value head j serves query heads
+    j*group .. j*group + group - 1."""
+    return np.repeat(_as64(x), group, axis=1)
+
+
+def attention_fwd_gqa_ref(q, k, v, scale, causal):
+    """Grouped-query (and multi-query) attention: Q has H heads, K and V have Hkv
+    heads with Hkv dividing H, and query head h attends with key/value head
+    h // (H / Hkv).  The attention variants named in "Atención Flash-2" (unite.ai
+    page); the definition is the standard attention of each query head with its
+    key/value head, so the oracle repeats K and V over the group.
+    """
+    group = q.shape[1] // k.shape[1]
+    assert group * k.shape[1] == q.shape[1]
+    return attention_fwd_ref(q, _repeat_heads(k, group), _repeat_heads(v, group), scale, causal)
+
+
+def attention_bwd_gqa_ref(q, k, v, do, scale, causal):
+    """Gradients of sum(O * dO) for grouped-query attention: dQ per query head;
+    dK and dV of a key/value head are the sums over its query heads (chain rule
+    through the repetition of K and V)."""
+    b_, hkv, n, d = np.shape(k)
+    group = q.shape[1] // hkv
+    dq, dk_e, dv_e = attention_bwd_ref(q, _repeat_heads(k, group), _repeat_heads(v, group), do, scale,
+                                       causal)
+    dk = dk_e.reshape(b_, hkv, group, n, d).sum(axis=2)
+    dv = dv_e.reshape(b_, hkv, group, n, d).sum(axis=2)
+    return dq, dk, dv

@@ -248,6 +248,43 @@ def test_backward_row_term_equals_rowsum_do_o():
     assert np.allclose((p * dp).sum(-1), (do * o).sum(-1), atol=1e-12)
 
 
+# --- grouped-query attention
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_backward_central_finite_differences(causal):
+    # H = 4 query heads sharing Hkv = 2 key/value heads: dK, dV must sum the group
+    n, d, sc, h = 5, 3, 0.8, 1e-6
+    q, k, v, do = rand(1, 4, n, d), rand(1, 2, n, d), rand(1, 2, n, d), rand(1, 4, n, d)
+    dq, dk, dv = orc.attention_bwd_gqa_ref(q, k, v, do, sc, causal)
+
+    def loss(q_, k_, v_):
+        o, _ = orc.attention_fwd_gqa_ref(q_, k_, v_, sc, causal)
+        return float(np.sum(o * do))
+
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            args = {"q": q, "k": k, "v": v}
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args[name] = xp
+            lp = loss(args["q"], args["k"], args["v"])
+            args[name] = xm
+            lm = loss(args["q"], args["k"], args["v"])
+            num[idx] = (lp - lm) / (2 * h)
+        assert np.linalg.norm(num - g) / np.linalg.norm(g) < 1e-6, name
+
+
+def test_gqa_single_group_is_plain_attention_per_head():
+    q, k, v = rand(2, 6, 20, 8), rand(2, 3, 20, 8), rand(2, 3, 20, 8)
+    o, lse = orc.attention_fwd_gqa_ref(q, k, v, 0.4, True)
+    for h in range(6):
+        o1, l1 = orc.attention_fwd_ref(q[:, h : h + 1], k[:, h // 2 : h // 2 + 1], v[:, h // 2 : h // 2 + 1], 0.4, True)
+        assert np.allclose(o[:, h : h + 1], o1, atol=1e-14) and np.allclose(lse[:, h : h + 1], l1, atol=1e-14)
+
+
 # --- stored regression fixture (written by tests/golden/make_golden.py, oracle only)
 
 

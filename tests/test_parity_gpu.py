@@ -198,3 +198,32 @@ def test_backward_config_2048_d128_causal_heads():
         sl = lambda x: to_f64(x)[b : b + 1, h : h + 1]
         ref = attention_bwd_ref(sl(q), sl(k), sl(v), sl(do), w.scale, w.causal)
         check_bwd(tuple(g[b : b + 1, h : h + 1] for g in got), ref, (b, h))
+
+
+# ---------------------------------------------------------------- grouped-query
+
+
+@pytest.mark.parametrize("H,Hkv", [(8, 2), (8, 1), (4, 4)])
+@pytest.mark.parametrize("N,causal,d", [(300, True, 128), (256, False, 64), (640, True, 64)])
+def test_gqa_forward_and_backward(H, Hkv, N, causal, d):
+    from exact_tiled_attention_35_b200.inputs import make_inputs
+    from oracle import attention_bwd_gqa_ref, attention_fwd_gqa_ref
+
+    q, _, _, do = make_inputs(1, H, N, d, seed=H * 10 + Hkv, with_do=True)
+    _, k, v = make_inputs(1, Hkv, N, d, seed=7 + Hkv)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = fa.forward_gqa(qd, kd, vd, causal=causal)
+    dq, dk, dv = fa.backward_gqa(qd, kd, vd, o, dod, lse, causal=causal)
+    fa.check_device_status()
+    scale = 1 / math.sqrt(d)
+    o_ref, lse_ref = attention_fwd_gqa_ref(to_f64(q), to_f64(k), to_f64(v), scale, causal)
+    check_fwd(to_f64(o), to_f64(lse), o_ref, lse_ref, (H, Hkv, N))
+    ref = attention_bwd_gqa_ref(to_f64(q), to_f64(k), to_f64(v), to_f64(do), scale, causal)
+    check_bwd(tuple(to_f64(x) for x in (dq, dk, dv)), ref, (H, Hkv, N))
+
+
+def test_gqa_with_full_heads_matches_multi_head_bitwise():
+    q, k, v = (t.cuda() for t in make_inputs(2, 4, 384, 128, seed=3))
+    o1, l1 = fa.forward(q, k, v, causal=True)
+    o2, l2 = fa.forward_gqa(q, k, v, causal=True)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
