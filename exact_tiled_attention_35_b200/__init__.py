@@ -34,6 +34,7 @@ SYMBOLS = {
     "fa_backward_gqa": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_fp32": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_noalloc": (_I, [_P] * 9 + [_I, _I, _I, _I, _F, _I, _P]),
+    "fa_debug_wait_timeout": (_I, [_P]),
     "fa_check_device_status": (_I, [_P]),
     "fa_last_error": (ctypes.c_char_p, []),
     "fa_status_string": (ctypes.c_char_p, [_I]),

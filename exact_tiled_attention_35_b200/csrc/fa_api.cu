@@ -159,6 +159,19 @@ fa_status backward_bf16(const void* q, const void* k, const void* v, const void*
 }  // namespace
 }  // namespace fa
 
+namespace fa {
+// One warp waits on an mbarrier that never completes; the bounded wait gives up,
+// records a timeout in the status word and the kernel returns.
+__global__ void wait_timeout_probe_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait(&bar, 0, 0xFF);
+  }
+}
+}  // namespace fa
+
 using namespace fa;
 
 extern "C" {
@@ -232,6 +245,11 @@ fa_status fa_backward_fp32(const float* q, const float* k, const float* v, const
   if (e != cudaSuccess) return FA_ERR_CUDA;
   return from_cuda(simt_backward(false, q, k, v, dout, lse, dsum, dq, dk, dv, BH, N, d, scale,
                                  causal ? 1 : 0, st));
+}
+
+fa_status fa_debug_wait_timeout(void* stream) {
+  fa::wait_timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  return from_cuda(cudaGetLastError());
 }
 
 fa_status fa_check_device_status(void* stream) {

@@ -130,6 +130,13 @@ fa_status fa_backward_noalloc(const void* q, const void* k, const void* v, const
                               const void* dout, const float* lse, void* dq, void* dk, void* dv,
                               int B, int H, int N, int d, float scale, int causal, void* stream);
 
+/* Diagnostic: launches one warp that waits on a barrier nothing ever completes,
+ * so the kernels' bounded wait runs out (after about 2 s) and records
+ * FA_ERR_DEVICE_TIMEOUT in the status word, then returns; the context stays
+ * usable.  Lets callers check their error path; not part of the attention
+ * computation (the pages have no counterpart).  Returns FA_OK once launched. */
+fa_status fa_debug_wait_timeout(void* stream);
+
 /* Synchronises `stream`, then reads and clears the current device's status
  * word.  FA_ERR_DEVICE_TIMEOUT if a kernel gave up a wait since the last call;
  * FA_ERR_CUDA if synchronisation failed; FA_OK otherwise. */
