@@ -81,6 +81,7 @@ struct Params {
   int N;
   int npairs;  // ceil(N / 256)
   int group;   // heads per scheduling group (their K/V stay resident in L2)
+  int items;   // work items = query-tile pairs x heads
   float scale;
   float scale_log2;
   int causal;
@@ -88,10 +89,11 @@ struct Params {
 
 struct Bars {
   uint64_t q_full[NQT];
+  uint64_t q_empty[NQT];  // the item's last S_t has read Q_t
   uint64_t s_full[NQT];
   uint64_t p_lo[NQT];   // probabilities of keys 0-63 of the tile in tensor memory
   uint64_t p_hi[NQT];   // keys 64-127
-  uint64_t o_full;
+  uint64_t o_full[NQT];   // the item's last P_t V has landed in O_t
   uint64_t drain;
   uint64_t kv_full[16];
   uint64_t kv_empty[16];
@@ -104,6 +106,22 @@ __device__ __forceinline__ int tiles_for(int q0, int N, int causal) {
   const int nkv = (N + BN - 1) / BN;
   if (!causal) return nkv;
   return min(nkv, q0 / BN + 1);
+}
+
+// Work item -> (query head, query-tile pair).  Under the causal mask the cost
+// of a pair grows with its index, so items run pair-major with the heaviest
+// pairs first; the snake walk below then gives every CTA a near-equal share.
+__device__ __forceinline__ void decode_item(const Params& p, int item, int& bh, int& pair) {
+  bh = item % p.BH;
+  const int rank = item / p.BH;
+  pair = p.causal ? (p.npairs - 1 - rank) : rank;
+}
+
+// The r-th item of this CTA: rounds of gridDim.x items, walked forwards in even
+// rounds and backwards in odd ones (a heavy item pairs with a light one).
+__device__ __forceinline__ int item_of(int r) {
+  const int g = gridDim.x;
+  return r * g + ((r & 1) ? (g - 1 - (int)blockIdx.x) : (int)blockIdx.x);
 }
 
 template <int D>
@@ -119,39 +137,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
-  // Blocks run in groups of p.group heads so that the K/V those CTAs share stay
-  // in L2; inside a group, heavy tiles come first under the causal mask (the
-  // pair index runs backwards).
-  const int blk = blockIdx.x;
-  const int full_blocks = (p.BH / p.group) * p.group * p.npairs;
-  int bh, rank;
-  if (blk < full_blocks) {
-    const int g = blk / (p.group * p.npairs), r = blk % (p.group * p.npairs);
-    bh = g * p.group + r % p.group;
-    rank = r / p.group;
-  } else {
-    const int gt = p.BH % p.group, r = blk - full_blocks;
-    bh = (p.BH / p.group) * p.group + r % gt;
-    rank = r / gt;
-  }
-  const int pair = p.causal ? (p.npairs - 1 - rank) : rank;
-  // key/value head of query head bh (grouped-query attention; bh itself when G = 1)
-  const int bkv = (bh / p.H) * (p.H / p.G) + (bh % p.H) / p.G;
-  const int qbase = pair * (NQT * BM);
-  int ntile[NQT];
+  // per item: query head, key/value head, first query row, key tiles per query tile
+  struct Item {
+    int bh, bkv, qbase, n[NQT], nmax;
+  };
+  auto item_info = [&](int item) {
+    Item it;
+    int pair;
+    decode_item(p, item, it.bh, pair);
+    // key/value head of query head bh (grouped-query attention; bh itself when G = 1)
+    it.bkv = (it.bh / p.H) * (p.H / p.G) + (it.bh % p.H) / p.G;
+    it.qbase = pair * (NQT * BM);
 #pragma unroll
-  for (int t = 0; t < NQT; ++t) ntile[t] = tiles_for(qbase + t * BM, p.N, p.causal);
-  const int nmax = max(ntile[0], ntile[1]);
+    for (int t = 0; t < NQT; ++t) it.n[t] = tiles_for(it.qbase + t * BM, p.N, p.causal);
+    it.nmax = max(it.n[0], it.n[1]);
+    return it;
+  };
 
   if (threadIdx.x == 0) {
 #pragma unroll
     for (int t = 0; t < NQT; ++t) {
       mbar_init(&bars->q_full[t], 1);
+      mbar_init(&bars->q_empty[t], 1);
+      mbar_init(&bars->o_full[t], 1);
       mbar_init(&bars->s_full[t], 1);
       mbar_init(&bars->p_lo[t], 128);
       mbar_init(&bars->p_hi[t], 128);
     }
-    mbar_init(&bars->o_full, 1);
     mbar_init(&bars->drain, 1);
     for (int s = 0; s < C::NSLOT; ++s) {
       mbar_init(&bars->kv_full[s], 1);
@@ -178,32 +190,42 @@ __global__ void __launch_bounds__(NTHREADS, 1)
    if (warp == kProducerWarp) {
     if (lane == 0) {
       bool ok = true;
-      for (int t = 0; t < NQT; ++t) {
-        if (ntile[t] == 0) continue;
-        mbar_arrive_expect_tx(&bars->q_full[t], C::TILE);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &mq, &bars->q_full[t], c * 64,
-                      qbase + t * BM, bh);
-      }
-      // ring sequence: K_0, V_0, K_1, V_1, ...
-      int issued = 0;
-      for (int seq = 0; seq < 2 * nmax && ok; ++seq) {
-        const int slot = seq % C::NSLOT, round = seq / C::NSLOT;
-        if (round > 0) ok = mbar_wait(&bars->kv_empty[slot], (round - 1) & 1, 1);
-        if (!ok) break;
-        const int j = seq >> 1;
-        const CUtensorMap* m = (seq & 1) ? &mv : &mk;
-        uint8_t* dst = sRing + slot * C::TILE;
-        mbar_arrive_expect_tx(&bars->kv_full[slot], C::TILE);
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(dst + c * C::CHUNK, m, &bars->kv_full[slot], c * 64, j * BN, bkv);
-        issued = seq + 1;
+      int gseq = 0;           // K/V ring position, continued across items
+      int qcnt[NQT] = {0, 0};  // Q_t loads so far
+      for (int r = 0; item_of(r) < p.items && ok; ++r) {
+        const Item w = item_info(item_of(r));
+        for (int t = 0; t < NQT && ok; ++t) {
+          if (w.n[t] == 0) continue;
+          if (qcnt[t] > 0) ok = mbar_wait(&bars->q_empty[t], (qcnt[t] - 1) & 1, 10);
+          if (!ok) break;
+          mbar_arrive_expect_tx(&bars->q_full[t], C::TILE);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &mq, &bars->q_full[t], c * 64,
+                        w.qbase + t * BM, w.bh);
+          ++qcnt[t];
+        }
+        // ring sequence: K_0, V_0, K_1, V_1, ...
+        for (int s2 = 0; s2 < 2 * w.nmax && ok; ++s2) {
+          const int seq = gseq + s2;
+          const int slot = seq % C::NSLOT, round = seq / C::NSLOT;
+          if (round > 0) ok = mbar_wait(&bars->kv_empty[slot], (round - 1) & 1, 1);
+          if (!ok) break;
+          const int j = s2 >> 1;
+          const CUtensorMap* m = (s2 & 1) ? &mv : &mk;
+          uint8_t* dst = sRing + slot * C::TILE;
+          mbar_arrive_expect_tx(&bars->kv_full[slot], C::TILE);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(dst + c * C::CHUNK, m, &bars->kv_full[slot], c * 64, j * BN, w.bkv);
+        }
+        gseq += 2 * w.nmax;
       }
       // make sure no copy into this CTA's shared memory is still in flight at exit
-      for (int s = 0; s < C::NSLOT && s < issued; ++s) {
-        const int last = s + ((issued - 1 - s) / C::NSLOT) * C::NSLOT;
-        mbar_wait(&bars->kv_full[s], (last / C::NSLOT) & 1, 2);
+      for (int slot = 0; slot < C::NSLOT && slot < gseq; ++slot) {
+        const int last = slot + ((gseq - 1 - slot) / C::NSLOT) * C::NSLOT;
+        mbar_wait(&bars->kv_full[slot], (last / C::NSLOT) & 1, 2);
       }
+      for (int t = 0; t < NQT; ++t)
+        if (qcnt[t] > 0) mbar_wait(&bars->q_full[t], (qcnt[t] - 1) & 1, 11);
     }
    } else if (warp == kMmaWarp) {
     if (lane == 0) {
@@ -212,8 +234,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       auto slot_of = [&](int seq) { return seq % C::NSLOT; };
       auto phase_of = [&](int seq) { return (uint32_t)((seq / C::NSLOT) & 1); };
       // S_t = Q_t K_j^T : A = Q_t (K-major), B = K_j (K-major), K = D in steps of 16
-      auto issue_s = [&](int t, int j) {
-        const uint32_t a0 = sq + t * C::TILE, b0 = sr + slot_of(2 * j) * C::TILE;
+      auto issue_s = [&](int t, int g0, int j) {
+        const uint32_t a0 = sq + t * C::TILE, b0 = sr + slot_of(g0 + 2 * j) * C::TILE;
         const uint32_t d_tmem = tmem + t * BN;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -224,8 +246,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       };
       // O_t += P_t V_j : A = P_t (tensor memory), B = V_j (MN-major), K = 128 keys,
       // issued in two halves (keys 0-63, 64-127) as the softmax group publishes them
-      auto issue_pv = [&](int t, int j, int half) {
-        const uint32_t b0 = sr + slot_of(2 * j + 1) * C::TILE;
+      auto issue_pv = [&](int t, int g0, int j, int half) {
+        const uint32_t b0 = sr + slot_of(g0 + 2 * j + 1) * C::TILE;
         const uint32_t d_tmem = tmem + 2 * BN + t * D;
         const uint32_t a_tmem = tmem + t * BN;
 #pragma unroll
@@ -233,47 +255,65 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b0 + kk * 16 * 128, C::CHUNK, 1024),
                  C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
       };
-      for (int t = 0; t < NQT && ok; ++t)
-        if (ntile[t] > 0) ok = mbar_wait(&bars->q_full[t], 0, 3);
-      if (ok && nmax > 0) ok = mbar_wait(&bars->kv_full[slot_of(0)], phase_of(0), 4);
-      if (ok) {
-        tc_fence_after();
-        for (int t = 0; t < NQT; ++t)
-          if (ntile[t] > 0) {
-            issue_s(t, 0);
-            mma_commit(&bars->s_full[t]);
-          }
-        if (nmax > 0) mma_commit(&bars->kv_empty[slot_of(0)]);
-      }
-      for (int j = 0; j < nmax && ok; ++j) {
-        ok = mbar_wait(&bars->kv_full[slot_of(2 * j + 1)], phase_of(2 * j + 1), 5);
-        bool k_next_ready = false;
-        for (int t = 0; t < NQT && ok; ++t) {
-          if (j >= ntile[t]) continue;
-          ok = mbar_wait(&bars->p_lo[t], j & 1, 6);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(t, j, 0);
-          ok = mbar_wait(&bars->p_hi[t], j & 1, 9);
-          if (!ok) break;
-          tc_fence_after();
-          issue_pv(t, j, 1);
-          if (j + 1 < ntile[t]) {
-            if (!k_next_ready) {
-              ok = mbar_wait(&bars->kv_full[slot_of(2 * j + 2)], phase_of(2 * j + 2), 7);
-              if (!ok) break;
-              tc_fence_after();
-              k_next_ready = true;
-            }
-            issue_s(t, j + 1);
-            mma_commit(&bars->s_full[t]);
-          }
-        }
+      int gseq = 0;                // K/V ring position of the item's K_0
+      int gt[NQT] = {0, 0};         // S_t tiles issued before this item
+      int qcnt[NQT] = {0, 0};       // items with a tile t before this one
+      for (int r = 0; item_of(r) < p.items && ok; ++r) {
+        const Item w = item_info(item_of(r));
+        for (int t = 0; t < NQT && ok; ++t)
+          if (w.n[t] > 0) ok = mbar_wait(&bars->q_full[t], qcnt[t] & 1, 3);
+        if (ok) ok = mbar_wait(&bars->kv_full[slot_of(gseq)], phase_of(gseq), 4);
         if (!ok) break;
-        mma_commit(&bars->kv_empty[slot_of(2 * j + 1)]);
-        if (k_next_ready) mma_commit(&bars->kv_empty[slot_of(2 * j + 2)]);
+        tc_fence_after();
+        // first S of the item; the previous item's last P_t V has already been
+        // issued, so overwriting S_t (where P_t lived) is ordered after it
+        for (int t = 0; t < NQT; ++t)
+          if (w.n[t] > 0) {
+            issue_s(t, gseq, 0);
+            mma_commit(&bars->s_full[t]);
+            if (w.n[t] == 1) mma_commit(&bars->q_empty[t]);
+          }
+        mma_commit(&bars->kv_empty[slot_of(gseq)]);
+        for (int j = 0; j < w.nmax && ok; ++j) {
+          ok = mbar_wait(&bars->kv_full[slot_of(gseq + 2 * j + 1)], phase_of(gseq + 2 * j + 1), 5);
+          bool k_next_ready = false;
+          for (int t = 0; t < NQT && ok; ++t) {
+            if (j >= w.n[t]) continue;
+            const uint32_t par = (uint32_t)((gt[t] + j) & 1);
+            // P of the item's first tile is published only after this softmax
+            // group has read the previous item's O_t, so the overwrite is safe
+            ok = mbar_wait(&bars->p_lo[t], par, 6);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(t, gseq, j, 0);
+            ok = mbar_wait(&bars->p_hi[t], par, 9);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(t, gseq, j, 1);
+            if (j + 1 < w.n[t]) {
+              if (!k_next_ready) {
+                ok = mbar_wait(&bars->kv_full[slot_of(gseq + 2 * j + 2)], phase_of(gseq + 2 * j + 2), 7);
+                if (!ok) break;
+                tc_fence_after();
+                k_next_ready = true;
+              }
+              issue_s(t, gseq, j + 1);
+              mma_commit(&bars->s_full[t]);
+              if (j + 2 == w.n[t]) mma_commit(&bars->q_empty[t]);  // last S_t of the item
+            } else {
+              mma_commit(&bars->o_full[t]);  // last P_t V of the item
+            }
+          }
+          if (!ok) break;
+          mma_commit(&bars->kv_empty[slot_of(gseq + 2 * j + 1)]);
+          if (k_next_ready) mma_commit(&bars->kv_empty[slot_of(gseq + 2 * j + 2)]);
+        }
+        gseq += 2 * w.nmax;
+        for (int t = 0; t < NQT; ++t) {
+          gt[t] += w.n[t];
+          qcnt[t] += w.n[t] > 0;
+        }
       }
-      if (ok) mma_commit(&bars->o_full);
       // wait for every MMA this thread issued before tensor memory is released
       mma_commit(&bars->drain);
       mbar_wait(&bars->drain, 0, 8);
@@ -284,16 +324,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // softmax / epilogue groups
     const int t = warp / 4;
     const int row = (warp % 4) * 32 + lane;
-    const int q_row = qbase + t * BM + row;
     const uint32_t lane_off = (uint32_t)((warp % 4) * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * BN;
     const uint32_t tO = tmem + lane_off + 2 * BN + t * D;
     const float c = p.scale_log2;
-    float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    const int n = ntile[t];
+    int gtile = 0, icnt = 0;  // S_t tiles and items with a tile t so far
+    for (int r = 0; item_of(r) < p.items && ok; ++r) {
+    const Item w = item_info(item_of(r));
+    const int n = w.n[t];
+    if (n == 0) continue;
+    const int bh = w.bh;
+    const int q_row = w.qbase + t * BM + row;
+    float m_used = -INFINITY, l = 0.f;
     for (int j = 0; j < n && ok; ++j) {
-      ok = mbar_wait(&bars->s_full[t], j & 1, 16 + t);
+      ok = mbar_wait(&bars->s_full[t], (gtile + j) & 1, 16 + t);
       if (!ok) break;
       tc_fence_after();
       float s[BN];
@@ -364,8 +409,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       f2_unpack(sum2[1], s2, s3);
       l = l * alpha + ((s0 + s1) + (s2 + s3));
     }
-    if (ok && n > 0) ok = mbar_wait(&bars->o_full, 0, 20 + t);
-    if (ok && n > 0) {
+    if (ok) ok = mbar_wait(&bars->o_full[t], icnt & 1, 20 + t);
+    if (ok) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (size_t)(q_row < p.N ? q_row : 0)) * D;
@@ -386,6 +431,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       if (q_row < p.N)
         p.lse[(size_t)bh * p.N + q_row] = l > 0.f ? m_used * p.scale + logf(l) : -INFINITY;
+    }
+    gtile += n;
+    ++icnt;
     }
   }
 
@@ -417,7 +465,12 @@ cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   p.scale = scale;
   p.scale_log2 = scale * fwd::kLog2e;
   p.causal = causal;
-  const dim3 grid((unsigned)(p.npairs * BH));
+  p.items = p.npairs * BH;
+  // persistent: one CTA per SM, each walking its share of the items
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const dim3 grid((unsigned)std::min(p.items, std::max(sms, 1)));
   cudaError_t e;
   if (d == 128) {
     const int smem = fwd::Cfg<128>::SMEM_BYTES;
