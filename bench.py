@@ -48,16 +48,19 @@ def algorithmic_flops(w, backward=None):
     return fwd, bwd
 
 
-KERNEL_SOURCES = ["exact_tiled_attention_35_b200/csrc/fa_device.cuh",
-                  "exact_tiled_attention_35_b200/csrc/fa_fwd_sm100.cu",
-                  "exact_tiled_attention_35_b200/csrc/fa_bwd_sm100.cu"]
+KERNEL_SOURCES = {
+    "fwd::fwd_kernel<128>": ["exact_tiled_attention_35_b200/csrc/fa_device.cuh",
+                             "exact_tiled_attention_35_b200/csrc/fa_fwd_sm100.cu"],
+    "bwd::main_kernel<128>": ["exact_tiled_attention_35_b200/csrc/fa_device.cuh",
+                              "exact_tiled_attention_35_b200/csrc/fa_bwd_sm100.cu"],
+}
 
 
-def kernel_source_hash():
+def kernel_source_hash(kernel):
     import hashlib
 
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
@@ -65,16 +68,16 @@ def kernel_source_hash():
 
 def profiled_traffic(kernel, workload):
     """DRAM bytes per launch of `kernel` on `workload` from profiles/traffic.json,
-    or None when absent or captured from different kernel sources."""
+    or None when absent or captured from other sources of that kernel."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(path):
+    if not os.path.exists(path) or kernel not in KERNEL_SOURCES:
         return None
     with open(path) as f:
         rec = json.load(f)
-    if rec.get("source_sha256") != kernel_source_hash():
-        return None
     entry = rec.get("kernels", {}).get(kernel)
     if not entry or entry.get("workload") != workload:
+        return None
+    if entry.get("source_sha256") != kernel_source_hash(kernel):
         return None
     return entry.get("dram_bytes_per_launch")
 

@@ -14,7 +14,9 @@
 // CTA layout (384 threads, registers rebalanced with setmaxnreg):
 //   warps 0-3  softmax + epilogue for query tile 0 (tensor-memory lanes 0-127)
 //   warps 4-7  softmax + epilogue for query tile 1
-//   warp  8    TMA producer: Q tiles once, then K_j, V_j into a ring of slots
+//   warp  8    TMA producer: draws the CTA's next work item when it has issued
+//              the loads of the current one, hands it to the other roles through
+//              a two-entry ring, then loads Q tiles and K_j, V_j into a ring of slots
 //   warp  9    tensor-memory allocator and MMA issuer (one elected thread)
 //   warps 10-11 idle (they complete the third warpgroup)
 // Tensor memory (512 columns): S_t at column 128*t (fp32 128x128, the bf16
@@ -36,6 +38,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "fa_device.cuh"
 #include "fa_kernels.h"
@@ -49,6 +52,9 @@ constexpr int NQT = 2;            // query tiles per CTA
 constexpr int NTHREADS = 384;  // three warpgroups
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kItemRing = 2;       // work items the producer may hand out ahead
+constexpr int kItemReaders = 9;    // MMA issuer and the 8 softmax warps
+constexpr int kSchedSlots = 256;   // ticket counters, one per launch in flight
 // Register split (setmaxnreg).  The launch gives every thread 168 registers,
 // 384 * 168 = 64512 in all; the shares sum to 128 * (2*208 + 88) = 64512.
 constexpr int kRegsSoftmax = 208;  // warpgroups 0 and 1
@@ -80,8 +86,9 @@ struct Params {
   int G;       // query heads per key/value head (1 without grouping)
   int N;
   int npairs;  // ceil(N / 256)
-  int group;   // heads per scheduling group (their K/V stay resident in L2)
+  int chunk;   // query heads per locality chunk (their K/V stay resident in L2)
   int items;   // work items = query-tile pairs x heads
+  int slot;    // ticket counter of this launch
   float scale;
   float scale_log2;
   int causal;
@@ -97,8 +104,19 @@ struct Bars {
   uint64_t drain;
   uint64_t kv_full[16];
   uint64_t kv_empty[16];
+  uint64_t it_full[kItemRing];   // the producer has written it_item[s]
+  uint64_t it_empty[kItemRing];  // every reader has taken it_item[s]
+  int it_item[kItemRing];
   uint32_t tmem_base;
 };
+
+// Ticket counters of the work-item scheduler: [slot][0] hands out work items past
+// the first gridDim.x, [slot][1] counts CTAs that have drawn their last ticket.
+// The last such CTA of a launch sets both back to zero, so the next launch that
+// draws the same slot starts clean.  The host draws slots round-robin; two launches in flight
+// at the same time on one device share a slot only if kSchedSlots launches were
+// issued in between.
+__device__ unsigned int g_fwd_tickets[kSchedSlots][2];
 
 // number of key tiles query tile starting at row q0 needs (0 if the tile is empty)
 __device__ __forceinline__ int tiles_for(int q0, int N, int causal) {
@@ -108,20 +126,18 @@ __device__ __forceinline__ int tiles_for(int q0, int N, int causal) {
   return min(nkv, q0 / BN + 1);
 }
 
-// Work item -> (query head, query-tile pair).  Under the causal mask the cost
-// of a pair grows with its index, so items run pair-major with the heaviest
-// pairs first; the snake walk below then gives every CTA a near-equal share.
+// Work item -> (query head, query-tile pair).  The heads are cut into chunks
+// whose K and V fit in L2 together; chunk by chunk, the items run pair-major,
+// and under the causal mask (where a pair's cost grows with its index) the
+// heaviest pairs come first.  CTAs take items in this order as they become
+// free, so the light pairs at the end of a chunk fill the gaps.
 __device__ __forceinline__ void decode_item(const Params& p, int item, int& bh, int& pair) {
-  bh = item % p.BH;
-  const int rank = item / p.BH;
+  const int per_chunk = p.chunk * p.npairs;
+  const int c = item / per_chunk, w = item - c * per_chunk;
+  const int h0 = c * p.chunk, hn = min(p.chunk, p.BH - h0);
+  const int rank = w / hn;
+  bh = h0 + (w - rank * hn);
   pair = p.causal ? (p.npairs - 1 - rank) : rank;
-}
-
-// The r-th item of this CTA: rounds of gridDim.x items, walked forwards in even
-// rounds and backwards in odd ones (a heavy item pairs with a light one).
-__device__ __forceinline__ int item_of(int r) {
-  const int g = gridDim.x;
-  return r * g + ((r & 1) ? (g - 1 - (int)blockIdx.x) : (int)blockIdx.x);
 }
 
 template <int D>
@@ -169,6 +185,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mbar_init(&bars->kv_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
+    for (int s = 0; s < kItemRing; ++s) {
+      mbar_init(&bars->it_full[s], 1);
+      mbar_init(&bars->it_empty[s], kItemReaders);
+    }
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -185,6 +205,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
+  // The k-th work item of this CTA from the producer's ring (>= p.items: none left).
+  auto take_item = [&](int k, int& item, int site) -> bool {
+    const int s = k % kItemRing;
+    if (!mbar_wait(&bars->it_full[s], (uint32_t)((k / kItemRing) & 1), site)) return false;
+    item = *reinterpret_cast<volatile int*>(&bars->it_item[s]);
+    return true;
+  };
+
   if (warp >= 8) {
    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
    if (warp == kProducerWarp) {
@@ -192,8 +220,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       bool ok = true;
       int gseq = 0;           // K/V ring position, continued across items
       int qcnt[NQT] = {0, 0};  // Q_t loads so far
-      for (int r = 0; item_of(r) < p.items && ok; ++r) {
-        const Item w = item_info(item_of(r));
+      unsigned int* tickets = &g_fwd_tickets[p.slot][0];
+      for (int r = 0; ok; ++r) {
+        // The first item of CTA b is b; each later one is drawn from the launch's
+        // ticket counter once this CTA's loads for the previous one are issued, so
+        // a CTA takes new work about when it is about to run out of it.
+        const int item = r == 0 ? (int)blockIdx.x : (int)gridDim.x + (int)atomicAdd(tickets, 1u);
+        const int s = r % kItemRing;
+        if (r >= kItemRing) ok = mbar_wait(&bars->it_empty[s], (uint32_t)((r / kItemRing - 1) & 1), 24);
+        if (!ok) break;
+        *reinterpret_cast<volatile int*>(&bars->it_item[s]) = item;
+        mbar_arrive(&bars->it_full[s]);
+        if (item >= p.items) break;
+        const Item w = item_info(item);
         for (int t = 0; t < NQT && ok; ++t) {
           if (w.n[t] == 0) continue;
           if (qcnt[t] > 0) ok = mbar_wait(&bars->q_empty[t], (qcnt[t] - 1) & 1, 10);
@@ -218,6 +257,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tma_load_3d(dst + c * C::CHUNK, m, &bars->kv_full[slot], c * 64, j * BN, w.bkv);
         }
         gseq += 2 * w.nmax;
+      }
+      // This CTA draws no more tickets (it has drawn one past the last item, or
+      // given up on a wait); the last CTA to get here resets the slot.
+      __threadfence();
+      if (atomicAdd(tickets + 1, 1u) == gridDim.x - 1) {
+        atomicExch(tickets, 0u);
+        atomicExch(tickets + 1, 0u);
       }
       // make sure no copy into this CTA's shared memory is still in flight at exit
       for (int slot = 0; slot < C::NSLOT && slot < gseq; ++slot) {
@@ -258,8 +304,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int gseq = 0;                // K/V ring position of the item's K_0
       int gt[NQT] = {0, 0};         // S_t tiles issued before this item
       int qcnt[NQT] = {0, 0};       // items with a tile t before this one
-      for (int r = 0; item_of(r) < p.items && ok; ++r) {
-        const Item w = item_info(item_of(r));
+      for (int r = 0; ok; ++r) {
+        int item = p.items;
+        ok = take_item(r, item, 25);
+        if (ok) mbar_arrive(&bars->it_empty[r % kItemRing]);
+        if (!ok || item >= p.items) break;
+        const Item w = item_info(item);
         for (int t = 0; t < NQT && ok; ++t)
           if (w.n[t] > 0) ok = mbar_wait(&bars->q_full[t], qcnt[t] & 1, 3);
         if (ok) ok = mbar_wait(&bars->kv_full[slot_of(gseq)], phase_of(gseq), 4);
@@ -330,8 +380,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const float c = p.scale_log2;
     bool ok = true;
     int gtile = 0, icnt = 0;  // S_t tiles and items with a tile t so far
-    for (int r = 0; item_of(r) < p.items && ok; ++r) {
-    const Item w = item_info(item_of(r));
+    for (int r = 0; ok; ++r) {
+    int item = p.items;
+    ok = take_item(r, item, 27);
+    __syncwarp();
+    if (ok && lane == 0) mbar_arrive(&bars->it_empty[r % kItemRing]);
+    if (!ok || item >= p.items) break;
+    const Item w = item_info(item);
     const int n = w.n[t];
     if (n == 0) continue;
     const int bh = w.bh;
@@ -445,6 +500,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
+// Query heads per locality chunk.  A chunk's K and V (4 N d bytes per key/value
+// head) should fit in about 40 MB of the 126 MB L2, a chunk should hold at least
+// two items per CTA so that its light tail balances the CTAs, chunks split the
+// heads evenly, and a group of query heads sharing a key/value head never
+// straddles two chunks.
+inline int chunk_heads(int BH, int G, int N, int d, int npairs, int grid) {
+  const long long kv_head = 4LL * N * d;
+  long long c = std::max(1LL, (40LL << 20) / kv_head) * G;
+  c = std::max<long long>(c, (2LL * grid + npairs - 1) / npairs);
+  c = std::min<long long>(((c + G - 1) / G) * G, BH);
+  const long long nch = (BH + c - 1) / c;
+  c = (BH + nch - 1) / nch;
+  c = std::min<long long>(((c + G - 1) / G) * G, BH);
+  return (int)c;
+}
+
 }  // namespace fwd
 
 cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
@@ -459,18 +530,18 @@ cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   p.G = H / Hkv;
   p.N = N;
   p.npairs = (N + 2 * fwd::BM - 1) / (2 * fwd::BM);
-  // heads whose K and V (4 N d bytes each) fit in about 48 MB of the 126 MB L2
-  const long long kv_bytes = 4LL * N * d;
-  p.group = (int)std::max(1LL, std::min<long long>(BH, (48LL << 20) / kv_bytes));
   p.scale = scale;
   p.scale_log2 = scale * fwd::kLog2e;
   p.causal = causal;
   p.items = p.npairs * BH;
-  // persistent: one CTA per SM, each walking its share of the items
+  // persistent: one CTA per SM, each taking items as it becomes free
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const dim3 grid((unsigned)std::min(p.items, std::max(sms, 1)));
+  p.chunk = fwd::chunk_heads(BH, p.G, N, d, p.npairs, (int)grid.x);
+  static std::atomic<unsigned int> launches{0};
+  p.slot = (int)(launches.fetch_add(1u, std::memory_order_relaxed) % fwd::kSchedSlots);
   cudaError_t e;
   if (d == 128) {
     const int smem = fwd::Cfg<128>::SMEM_BYTES;

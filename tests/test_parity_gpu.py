@@ -137,6 +137,42 @@ def test_forward_is_deterministic():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("B,H,N,d,causal", [(2, 32, 4096, 128, True), (1, 12, 16384, 64, True),
+                                             (1, 7, 32768, 64, True), (4, 16, 1024, 64, False)])
+def test_forward_schedule_covers_every_item_once(B, H, N, d, causal):
+    # The persistent forward hands (head, query-tile pair) items to CTAs through
+    # a ticket counter, in L2-sized head chunks.  Each item's arithmetic does not
+    # depend on which CTA runs it or when, so the whole launch must equal, bit
+    # for bit, launches of one head each (a single chunk, a different order), and
+    # a second whole launch (a different dynamic assignment).
+    q, k, v = (t.cuda() for t in make_inputs(B, H, N, d, seed=21))
+    o, lse = fa.forward(q, k, v, causal=causal)
+    o2, lse2 = fa.forward(q, k, v, causal=causal)
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+    for b in range(B):
+        for h in range(H):
+            sl = (slice(b, b + 1), slice(h, h + 1))
+            oh, lh = fa.forward(q[sl].contiguous(), k[sl].contiguous(), v[sl].contiguous(), causal=causal)
+            assert torch.equal(oh, o[sl]) and torch.equal(lh, lse[sl]), (b, h)
+    fa.check_device_status()
+
+
+def test_forward_ticket_slots_reset_across_many_launches():
+    # More launches than the scheduler has ticket slots: every slot is reused, so a
+    # slot left dirty by a previous launch would make CTAs skip items.
+    q, k, v = (t.cuda() for t in make_inputs(1, 6, 1000, 64, seed=22))
+    o0, l0 = fa.forward(q, k, v, causal=True)
+    o = torch.empty_like(o0)
+    lse = torch.empty_like(l0)
+    bad = torch.zeros((), dtype=torch.bool, device="cuda")
+    for _ in range(600):
+        o.fill_(float("nan"))
+        fa.forward(q, k, v, causal=True, out=o, lse=lse)
+        bad |= (o != o0).any() | (lse != l0).any()
+    assert not bool(bad)
+    fa.check_device_status()
+
+
 def test_forward_key_shift_invariance_on_gpu():
     # adding one vector u to every key leaves O unchanged (the LSE shift is checked
     # against the oracle on the shifted keys)
