@@ -264,38 +264,41 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
    } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      const uint32_t uK = smem_u32(sK), uV = smem_u32(sV), uDS = smem_u32(sDS);
-      auto stage_q = [&](int it) { return smem_u32(smem + C::OFF_Q + (it % NST) * C::TILE); };
-      const uint32_t udO = smem_u32(smem + C::OFF_DO);
+      // One descriptor for the start of shared memory (the K tile, K-major); every
+      // operand is a compile-time offset from it (one add per MMA), a Q stage a
+      // per-tile one, and an MN-major operand differs only in LBO.
+      const uint64_t d0 = sdesc_sw128(smem_u32(smem), 16, 1024);
+      constexpr uint64_t kToMn = (uint64_t)((C::CHUNK >> 4) - 1) << 16;  // LBO 16 B -> CHUNK
+      auto q_desc = [&](int it) { return sdesc_at(opaque(d0), C::OFF_Q + (it % NST) * C::TILE); };
       // S^T = K Q^T  (keys x queries), K = d
       auto issue_s = [&](int it) {
-        const uint32_t uQ = stage_q(it);
+        const uint64_t dq = q_desc(it), dk = opaque(d0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_ss(tmem + C::T_S, sdesc_sw128(uK + ko, 16, 1024), sdesc_sw128(uQ + ko, 16, 1024),
-                 C::IDESC_S, kk > 0);
+          mma_ss(tmem + C::T_S, sdesc_at(dk, C::OFF_K + ko), sdesc_at(dq, ko), C::IDESC_S, kk > 0);
         }
         mma_commit(&bars->s_full);
       };
       // dP^T = V dO^T
       auto issue_dp = [&](int it) {
+        const uint64_t d = opaque(d0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_ss(tmem + C::T_DP, sdesc_sw128(uV + ko, 16, 1024), sdesc_sw128(udO + ko, 16, 1024),
-                 C::IDESC_S, kk > 0);
+          mma_ss(tmem + C::T_DP, sdesc_at(d, C::OFF_V + ko), sdesc_at(d, C::OFF_DO + ko), C::IDESC_S,
+                 kk > 0);
         }
         mma_commit(&bars->dp_full);
       };
       // dV += P^T dO  (keys x d), K = 128 queries, P^T from tensor memory (queries
       // 64h .. 64h+63 packed at column 64h)
       auto issue_dv = [&](int it) {
+        const uint64_t d = opaque(d0) + kToMn;
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk)
           mma_ts(tmem + C::T_DV, tmem + C::T_S + 64 * (kk / 4) + 8 * (kk % 4),
-                 sdesc_sw128(udO + kk * 2048, C::CHUNK, 1024), C::IDESC_DKV,
-                 (it > 0 || kk > 0) ? 1u : 0u);
+                 sdesc_at(d, C::OFF_DO + kk * 2048), C::IDESC_DKV, (it > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&bars->do_empty);
       };
       // Order per query tile i (after the prologue S(0), dP(0)):
@@ -316,7 +319,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       for (int it = 0; it < niter && ok; ++it) {
         const int st = it % NST;
-        const uint32_t uQ = stage_q(it);
         const bool more = it + 1 < niter;
         ok = mbar_wait(&bars->p_full, it & 1, 46);
         if (!ok) break;
@@ -332,17 +334,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (!ok) break;
         tc_fence_after();
         // dQ_part = dS K  (queries x d), K = 128 keys; written over dP^T
+        const uint64_t dmn = opaque(d0) + kToMn;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ss(tmem + C::T_DP, sdesc_sw128(uDS + kk * 2048, C::CHUNK, 1024),
-                 sdesc_sw128(uK + kk * 2048, C::CHUNK, 1024), C::IDESC_DQ, kk > 0);
+          mma_ss(tmem + C::T_DP, sdesc_at(dmn, C::OFF_DS + kk * 2048), sdesc_at(dmn, C::OFF_K + kk * 2048),
+                 C::IDESC_DQ, kk > 0);
         mma_commit(&bars->dq_full);
         // dK += dS^T Q  (keys x d), K = 128 queries
+        const uint64_t dq_mn = q_desc(it) + kToMn, dds = opaque(d0);
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_ss(tmem + C::T_DK, sdesc_sw128(uDS + ko, 16, 1024),
-                 sdesc_sw128(uQ + kk * 2048, C::CHUNK, 1024), C::IDESC_DKV,
+          mma_ss(tmem + C::T_DK, sdesc_at(dds, C::OFF_DS + ko), sdesc_at(dq_mn, kk * 2048), C::IDESC_DKV,
                  (it > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(&bars->ds_free);

@@ -202,6 +202,17 @@ __device__ __forceinline__ void tmem_ld16x256b_x8(uint32_t taddr, uint32_t (&r)[
       : "r"(taddr));
 }
 
+// 32 lanes x 16 columns of 32 bits, one lane per thread of the warp.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -224,6 +235,22 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// The same descriptor for an operand `bytes` further on in shared memory.  The
+// start-address field is the low 14 bits (address >> 4, below 256 KB), so the
+// move is one add; with a compile-time offset it costs the MMA issuer a single
+// instruction where rebuilding the descriptor costs several.
+__device__ __forceinline__ uint64_t sdesc_at(uint64_t desc, uint32_t bytes) {
+  return desc + (uint64_t)(bytes >> 4);
+}
+
+// Hides a value's origin from the compiler so that descriptors derived from it
+// inside a loop are formed there (one add each) rather than hoisted out of the
+// loop into dozens of live registers.
+__device__ __forceinline__ uint64_t opaque(uint64_t v) {
+  asm volatile("" : "+l"(v));
+  return v;
 }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.

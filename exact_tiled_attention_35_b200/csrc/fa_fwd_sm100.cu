@@ -276,32 +276,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
    } else if (warp == kMmaWarp) {
     if (lane == 0) {
       bool ok = true;
-      const uint32_t sq = smem_u32(sQ), sr = smem_u32(sRing);
-      auto slot_of = [&](int seq) { return seq % C::NSLOT; };
-      auto phase_of = [&](int seq) { return (uint32_t)((seq / C::NSLOT) & 1); };
+      // Descriptors are built once; each MMA moves them by a compile-time offset
+      // (one add), and ring positions advance incrementally, so the issuing thread
+      // spends few instructions per MMA.
+      // One descriptor for the start of shared memory (Q_0, K-major); the ring
+      // follows the Q tiles, and an MN-major operand differs only in LBO.
+      const uint64_t d0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      constexpr uint64_t kToMn = (uint64_t)((C::CHUNK >> 4) - 1) << 16;  // LBO 16 B -> CHUNK
       // S_t = Q_t K_j^T : A = Q_t (K-major), B = K_j (K-major), K = D in steps of 16
-      auto issue_s = [&](int t, int g0, int j) {
-        const uint32_t a0 = sq + t * C::TILE, b0 = sr + slot_of(g0 + 2 * j) * C::TILE;
+      auto issue_s = [&](int t, uint32_t kslot) {
+        const uint64_t d = opaque(d0);
+        const uint64_t a = sdesc_at(d, t * C::TILE), b = sdesc_at(d, C::SMEM_Q + kslot * C::TILE);
         const uint32_t d_tmem = tmem + t * BN;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_ss(d_tmem, sdesc_sw128(a0 + koff, 16, 1024), sdesc_sw128(b0 + koff, 16, 1024),
-                 C::IDESC_QK, kk > 0);
+          mma_ss(d_tmem, sdesc_at(a, koff), sdesc_at(b, koff), C::IDESC_QK, kk > 0);
         }
       };
       // O_t += P_t V_j : A = P_t (tensor memory), B = V_j (MN-major), K = 128 keys,
       // issued in two halves (keys 0-63, 64-127) as the softmax group publishes them
-      auto issue_pv = [&](int t, int g0, int j, int half) {
-        const uint32_t b0 = sr + slot_of(g0 + 2 * j + 1) * C::TILE;
+      auto issue_pv = [&](int t, uint32_t vslot, int j, int half) {
+        const uint64_t b = sdesc_at(opaque(d0), C::SMEM_Q + vslot * C::TILE) + kToMn;
         const uint32_t d_tmem = tmem + 2 * BN + t * D;
         const uint32_t a_tmem = tmem + t * BN;
 #pragma unroll
-        for (int kk = half * 4; kk < half * 4 + 4; ++kk)
-          mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(b0 + kk * 16 * 128, C::CHUNK, 1024),
-                 C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int q = 0; q < 4; ++q) {
+          const int kk = half * 4 + q;
+          mma_ts(d_tmem, a_tmem + kk * 8, sdesc_at(b, kk * 16 * 128), C::IDESC_PV,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+        }
       };
-      int gseq = 0;                // K/V ring position of the item's K_0
+      auto advance = [](uint32_t& slot, uint32_t& phase) {
+        if (++slot == (uint32_t)C::NSLOT) {
+          slot = 0;
+          phase ^= 1u;
+        }
+      };
+      uint32_t kslot = 0, kphase = 0;  // ring position of the next K tile (the item's K_0)
       int gt[NQT] = {0, 0};         // S_t tiles issued before this item
       int qcnt[NQT] = {0, 0};       // items with a tile t before this one
       for (int r = 0; ok; ++r) {
@@ -312,20 +324,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const Item w = item_info(item);
         for (int t = 0; t < NQT && ok; ++t)
           if (w.n[t] > 0) ok = mbar_wait(&bars->q_full[t], qcnt[t] & 1, 3);
-        if (ok) ok = mbar_wait(&bars->kv_full[slot_of(gseq)], phase_of(gseq), 4);
+        if (ok) ok = mbar_wait(&bars->kv_full[kslot], kphase, 4);
         if (!ok) break;
         tc_fence_after();
         // first S of the item; the previous item's last P_t V has already been
         // issued, so overwriting S_t (where P_t lived) is ordered after it
         for (int t = 0; t < NQT; ++t)
           if (w.n[t] > 0) {
-            issue_s(t, gseq, 0);
+            issue_s(t, kslot);
             mma_commit(&bars->s_full[t]);
             if (w.n[t] == 1) mma_commit(&bars->q_empty[t]);
           }
-        mma_commit(&bars->kv_empty[slot_of(gseq)]);
+        mma_commit(&bars->kv_empty[kslot]);
         for (int j = 0; j < w.nmax && ok; ++j) {
-          ok = mbar_wait(&bars->kv_full[slot_of(gseq + 2 * j + 1)], phase_of(gseq + 2 * j + 1), 5);
+          uint32_t vslot = kslot, vphase = kphase;
+          advance(vslot, vphase);  // V_j
+          uint32_t nslot = vslot, nphase = vphase;
+          advance(nslot, nphase);  // K_{j+1} (the next item's K_0 after the last j)
+          ok = mbar_wait(&bars->kv_full[vslot], vphase, 5);
           bool k_next_ready = false;
           for (int t = 0; t < NQT && ok; ++t) {
             if (j >= w.n[t]) continue;
@@ -335,19 +351,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             ok = mbar_wait(&bars->p_lo[t], par, 6);
             if (!ok) break;
             tc_fence_after();
-            issue_pv(t, gseq, j, 0);
+            issue_pv(t, vslot, j, 0);
             ok = mbar_wait(&bars->p_hi[t], par, 9);
             if (!ok) break;
             tc_fence_after();
-            issue_pv(t, gseq, j, 1);
+            issue_pv(t, vslot, j, 1);
             if (j + 1 < w.n[t]) {
               if (!k_next_ready) {
-                ok = mbar_wait(&bars->kv_full[slot_of(gseq + 2 * j + 2)], phase_of(gseq + 2 * j + 2), 7);
+                ok = mbar_wait(&bars->kv_full[nslot], nphase, 7);
                 if (!ok) break;
                 tc_fence_after();
                 k_next_ready = true;
               }
-              issue_s(t, gseq, j + 1);
+              issue_s(t, nslot);
               mma_commit(&bars->s_full[t]);
               if (j + 2 == w.n[t]) mma_commit(&bars->q_empty[t]);  // last S_t of the item
             } else {
@@ -355,10 +371,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
           }
           if (!ok) break;
-          mma_commit(&bars->kv_empty[slot_of(gseq + 2 * j + 1)]);
-          if (k_next_ready) mma_commit(&bars->kv_empty[slot_of(gseq + 2 * j + 2)]);
+          mma_commit(&bars->kv_empty[vslot]);
+          if (k_next_ready) mma_commit(&bars->kv_empty[nslot]);
+          kslot = nslot;
+          kphase = nphase;
         }
-        gseq += 2 * w.nmax;
         for (int t = 0; t < NQT; ++t) {
           gt[t] += w.n[t];
           qcnt[t] += w.n[t] > 0;
