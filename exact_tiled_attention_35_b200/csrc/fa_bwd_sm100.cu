@@ -93,6 +93,7 @@ struct Params {
   int N;
   int Npad;
   int nkv;             // number of key tiles = Npad / 128
+  int chunk;           // key/value heads per locality chunk
   float scale;
   float scale_log2;
   int causal;
@@ -174,10 +175,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // heavy key tiles first under the causal mask (tile j sees query tiles j..)
+  // CTA -> (key/value head, key tile).  The heads are cut into chunks whose
+  // K, V, Q, dO and fp32 dQ accumulator fit in L2 together; chunk by chunk,
+  // CTAs run key-tile-major with the heavy tiles first under the causal mask
+  // (tile j sees query tiles j..), and the block scheduler hands them to SMs in
+  // that order as SMs free up.
   const int blk = blockIdx.x;
-  const int bkv = blk % p.BHkv;  // key/value head
-  const int j = blk / p.BHkv;
+  const int per_chunk = p.chunk * p.nkv;
+  const int chunk_id = blk / per_chunk, w_in = blk - chunk_id * per_chunk;
+  const int h0 = chunk_id * p.chunk, hn = min(p.chunk, p.BHkv - h0);
+  const int j = w_in / hn;
+  const int bkv = h0 + (w_in - j * hn);  // key/value head
   const int nq = p.nkv;
   const int i0 = p.causal ? j : 0;
   const int nqi = nq - i0;        // query tiles per query head
@@ -598,6 +606,21 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict
   }
 }
 
+// Key/value heads per locality chunk.  Per key/value head the pass touches
+// K and V (4 N d bytes), the Q and dO of its G query heads (4 G N d bytes) and
+// their fp32 dQ accumulator (4 G N d bytes), which the reduce-adds must find in
+// L2; a chunk keeps that near 80 MB of the 126 MB L2.  A chunk also holds at
+// least two waves of CTAs so that its light tail balances the SMs, and chunks
+// split the heads evenly.
+inline int chunk_heads(int BHkv, int G, int N, int d, int nkv, int sms) {
+  const long long per_head = 4LL * N * d * (2LL * G + 1);
+  long long c = std::max(1LL, (80LL << 20) / per_head);
+  c = std::max<long long>(c, (2LL * sms + nkv - 1) / nkv);
+  c = std::min<long long>(c, BHkv);
+  const long long nch = (BHkv + c - 1) / c;
+  return (int)((BHkv + nch - 1) / nch);
+}
+
 }  // namespace bwd
 
 size_t sm100_backward_workspace(int BH, int N, int d) {
@@ -650,6 +673,10 @@ cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const C
   p.scale = scale;
   p.scale_log2 = scale * bwd::kLog2e;
   p.causal = causal;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  p.chunk = bwd::chunk_heads(p.BHkv, p.G, N, d, p.nkv, std::max(sms, 1));
   const dim3 grid((unsigned)(p.nkv * p.BHkv));
   if (d == 128) {
     const int smem = bwd::Cfg<128>::SMEM_BYTES;
