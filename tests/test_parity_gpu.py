@@ -236,6 +236,32 @@ def test_backward_config_2048_d128_causal_heads():
         check_bwd(tuple(g[b : b + 1, h : h + 1] for g in got), ref, (b, h))
 
 
+@pytest.mark.parametrize("B,H,Hkv,N,d,causal", [(2, 16, 16, 2048, 128, True), (2, 32, 32, 4096, 128, True),
+                                                 (1, 24, 6, 4096, 64, True), (1, 8, 8, 8192, 128, False)])
+def test_backward_schedule_covers_every_tile_once(B, H, Hkv, N, d, causal):
+    # The backward runs its (key/value head, key tile) CTAs in L2-sized head
+    # chunks.  dK and dV of a key tile come from one CTA whatever the order, so
+    # a multi-chunk launch must give them bit for bit as launches of one
+    # key/value head each do; dQ is summed by reduce-adds in an order that
+    # varies, so it is held to fp32 rounding.
+    q, k, v, do = (t.cuda() for t in make_inputs(B, H, N, d, seed=23, with_do=True))
+    k, v = k[:, :Hkv].contiguous(), v[:, :Hkv].contiguous()
+    o, lse = fa.forward_gqa(q, k, v, causal=causal)
+    dq, dk, dv = fa.backward_gqa(q, k, v, o, do, lse, causal=causal)
+    G = H // Hkv
+    for b in range(B):
+        for hk in range(Hkv):
+            qs = (slice(b, b + 1), slice(hk * G, (hk + 1) * G))
+            ks = (slice(b, b + 1), slice(hk, hk + 1))
+            dq1, dk1, dv1 = fa.backward_gqa(q[qs].contiguous(), k[ks].contiguous(), v[ks].contiguous(),
+                                            o[qs].contiguous(), do[qs].contiguous(), lse[qs].contiguous(),
+                                            causal=causal)
+            assert torch.equal(dk1, dk[ks]) and torch.equal(dv1, dv[ks]), (b, hk)
+            rel = float((dq1.float() - dq[qs].float()).norm() / dq1.float().norm())
+            assert rel < 1e-3, (b, hk, rel)
+    fa.check_device_status()
+
+
 # ---------------------------------------------------------------- grouped-query
 
 
