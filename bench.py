@@ -242,7 +242,8 @@ def run_reference(args, w, world, rank):
                                         "causal": w.causal, "l2": "n/a (CPU)"},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)),
                          "kind": "oracle",
-                         "sample": f"one (b,h) head of {w.name} per step (fwd+bwd fp64, full N x N)"},
+                         "sample": f"one (b,h) head of {w.name} per step ({'fwd+bwd' if w.backward else 'fwd'} "
+                                   f"fp64, full N x N)"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -388,8 +389,8 @@ def run_ours(args, w, world, rank, local):
     if rank == 0 and world == 1 and not args.skip_cpu:
         f, el, heads, cores = oracle_sample(w, args.cpu_budget)
         cpu = {"value": f / el / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-               "sample": f"{heads} (b,h) head(s) of {w.name}, fwd+bwd in fp64 with the full N x N "
-                         f"matrix, {el:.1f} s"}
+               "sample": f"{heads} (b,h) head(s) of {w.name}, {'fwd+bwd' if w.backward else 'fwd'} in fp64 "
+                         f"with the full N x N matrix, {el:.1f} s"}
 
     if rank == 0:
         line = {
