@@ -28,7 +28,14 @@ Not on the pages, taken from the method's statement of the task: the causal mask
 log-sum-exp output (natural log, of the scaled scores) and the backward pass
 (the closed-form softmax Jacobian).
 
-All arrays are numpy float64 with layout [B, H, N, d] (LSE: [B, H, N]).
+Reading for unequal query and key lengths (Nq queries, Nk keys), which the pages
+do not treat: the causal mask is aligned at the bottom right, key j visible to
+query i iff j <= i + (Nk - Nq), so the last query sees every key and Nq = Nk is
+the square mask above.  A query that sees no key (i < Nq - Nk) has O = 0 and
+LSE = -inf.
+
+All arrays are numpy float64 with layout [B, H, N, d] (LSE: [B, H, N]); K and V
+may have their own length Nk.
 """
 
 from __future__ import annotations
@@ -90,16 +97,31 @@ def scores(q, k, scale, causal):
     """S = scale * Q K^T per (batch, head), with the causal mask applied.
 
     The score tensor of the standard-attention listing (unite.ai page), here
-    one [N, N] matrix per (b, h).  Masked entries are -inf.
+    one [Nq, Nk] matrix per (b, h).  Masked entries are -inf: under the causal
+    mask, key j is hidden from query i when j > i + (Nk - Nq).
     """
     q = _as64(q)
     k = _as64(k)
     s = scale * np.matmul(q, np.swapaxes(k, -1, -2))
     if causal:
-        n = q.shape[2]
-        above = np.triu(np.ones((n, n), dtype=bool), k=1)
+        nq, nk = q.shape[2], k.shape[2]
+        above = np.triu(np.ones((nq, nk), dtype=bool), k=nk - nq + 1)
         s = np.where(above, -np.inf, s)
     return s
+
+
+def _softmax_rows(s):
+    """Row-wise safe softmax of a score tensor and its log-sum-exp; a row with no
+    visible key gets probabilities 0 and LSE -inf."""
+    m = np.max(s, axis=-1, keepdims=True)
+    empty = np.isneginf(m)
+    m0 = np.where(empty, 0.0, m)
+    e = np.exp(s - m0)
+    l = np.sum(e, axis=-1, keepdims=True)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        p = np.where(empty, 0.0, e / np.where(empty, 1.0, l))
+        lse = np.where(empty, -np.inf, m0 + np.log(np.where(empty, 1.0, l)))
+    return p, lse[..., 0]
 
 
 def attention_fwd_ref(q, k, v, scale, causal):
@@ -110,12 +132,9 @@ def attention_fwd_ref(q, k, v, scale, causal):
     exp(S_ij - m_i) with m_i the row maximum (safe softmax).
     """
     v = _as64(v)
-    s = scores(q, k, scale, causal)
-    m = np.max(s, axis=-1, keepdims=True)
-    lse = m + np.log(np.sum(np.exp(s - m), axis=-1, keepdims=True))
-    p = np.exp(s - lse)
+    p, lse = _softmax_rows(scores(q, k, scale, causal))
     o = np.matmul(p, v)
-    return o, lse[..., 0]
+    return o, lse
 
 
 def attention_bwd_ref(q, k, v, do, scale, causal):
@@ -133,10 +152,7 @@ def attention_bwd_ref(q, k, v, do, scale, causal):
     k = _as64(k)
     v = _as64(v)
     do = _as64(do)
-    s = scores(q, k, scale, causal)
-    m = np.max(s, axis=-1, keepdims=True)
-    e = np.exp(s - m)
-    p = e / np.sum(e, axis=-1, keepdims=True)
+    p, _ = _softmax_rows(scores(q, k, scale, causal))
     dv = np.matmul(np.swapaxes(p, -1, -2), do)
     dp = np.matmul(do, np.swapaxes(v, -1, -2))
     ds = p * (dp - np.sum(p * dp, axis=-1, keepdims=True))
@@ -150,14 +166,16 @@ def attention_rows_ref(q, k, v, rows, scale, causal):
 
     Same definition as ``attention_fwd_ref``, evaluated row by row: for each
     (b, h) and each query index i in ``rows[h]`` (or ``rows`` when it is one
-    list for all heads) the score row S[i, :] (keys 0..i when causal) is formed,
-    then its safe softmax and the weighted sum of V.
+    list for all heads) the score row S[i, :] (keys 0..i + Nk - Nq when causal)
+    is formed, then its safe softmax and the weighted sum of V.  A row with no
+    visible key gets O = 0 and LSE = -inf.
     Returns (o [B, H, R, d], lse [B, H, R]).
     """
     q = _as64(q)
     k = _as64(k)
     v = _as64(v)
     b_, h_, n, d = q.shape
+    off = k.shape[2] - n
     per_head = isinstance(rows, (list, tuple)) and len(rows) > 0 and np.ndim(rows[0]) == 1
     r = len(rows[0]) if per_head else len(rows)
     o = np.zeros((b_, h_, r, d))
@@ -167,8 +185,12 @@ def attention_rows_ref(q, k, v, rows, scale, causal):
             sel = rows[h] if per_head else rows
             for t, i in enumerate(sel):
                 i = int(i)
-                kk = k[b, h, : i + 1] if causal else k[b, h]
-                vv = v[b, h, : i + 1] if causal else v[b, h]
+                last = i + off + 1 if causal else k.shape[2]
+                if last <= 0:
+                    lse[b, h, t] = -np.inf
+                    continue
+                kk = k[b, h, :last]
+                vv = v[b, h, :last]
                 srow = scale * (kk @ q[b, h, i])
                 m = np.max(srow)
                 e = np.exp(srow - m)
@@ -192,6 +214,7 @@ def online_softmax_attention(q, k, v, scale, causal, block_q=128, block_k=128):
     k = _as64(k)
     v = _as64(v)
     b_, h_, n, d = q.shape
+    nk = k.shape[2]
     o = np.zeros_like(q)
     lse = np.zeros((b_, h_, n))
     for b in range(b_):
@@ -202,13 +225,13 @@ def online_softmax_attention(q, k, v, scale, causal, block_q=128, block_k=128):
                 ob = np.zeros((i1 - i0, d))
                 mrow = np.full((i1 - i0, 1), -np.inf)
                 lrow = np.zeros((i1 - i0, 1))
-                for j0 in range(0, n, block_k):
-                    j1 = min(n, j0 + block_k)
+                for j0 in range(0, nk, block_k):
+                    j1 = min(nk, j0 + block_k)
                     sb = scale * (qb @ k[b, h, j0:j1].T)
                     if causal:
                         qi = np.arange(i0, i1)[:, None]
                         kj = np.arange(j0, j1)[None, :]
-                        sb = np.where(kj > qi, -np.inf, sb)
+                        sb = np.where(kj > qi + (nk - n), -np.inf, sb)
                     m_new = np.maximum(mrow, np.max(sb, axis=-1, keepdims=True))
                     # a row whose max is still -inf has seen no visible key yet
                     safe_m = np.where(np.isneginf(m_new), 0.0, m_new)
@@ -221,7 +244,8 @@ def online_softmax_attention(q, k, v, scale, causal, block_q=128, block_k=128):
                         )
                     mrow, lrow = m_new, l_new
                 o[b, h, i0:i1] = ob
-                lse[b, h, i0:i1] = (mrow + np.log(lrow))[:, 0]
+                with np.errstate(divide="ignore"):
+                    lse[b, h, i0:i1] = np.where(lrow > 0, mrow + np.log(np.where(lrow > 0, lrow, 1.0)), -np.inf)[:, 0]
     return o, lse
 
 

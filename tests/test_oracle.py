@@ -374,3 +374,114 @@ def test_planted_backward_slip_is_caught():
         qm[idx] -= h
         num[idx] = (_loss(qp, k, v, do, sc, False) - _loss(qm, k, v, do, sc, False)) / (2 * h)
     assert np.linalg.norm(num - dq_bad) / np.linalg.norm(num) > 1e-3
+
+
+# --- unequal query and key lengths (Nq != Nk); causal mask aligned bottom right
+
+
+@pytest.mark.parametrize("nq,nk", [(3, 5), (5, 3), (1, 4), (4, 1), (6, 6)])
+def test_unequal_lengths_pure_python_brute_force(nq, nk):
+    d, sc = 3, 0.7
+    q, k, v = rand(1, 1, nq, d), rand(1, 1, nk, d), rand(1, 1, nk, d)
+    o, lse = orc.attention_fwd_ref(q, k, v, sc, True)
+    for i in range(nq):
+        keys = [j for j in range(nk) if j <= i + nk - nq]
+        if not keys:  # no visible key: O = 0, LSE = -inf
+            assert lse[0, 0, i] == -np.inf and np.all(o[0, 0, i] == 0.0)
+            continue
+        w = {j: math.exp(sc * sum(q[0, 0, i, c] * k[0, 0, j, c] for c in range(d))) for j in keys}
+        z = sum(w.values())
+        assert math.isclose(lse[0, 0, i], math.log(z), rel_tol=1e-13, abs_tol=1e-13)
+        for c in range(d):
+            ref = sum(w[j] * v[0, 0, j, c] for j in keys) / z
+            assert math.isclose(o[0, 0, i, c], ref, rel_tol=1e-12, abs_tol=1e-13)
+
+
+def test_fewer_queries_are_the_last_rows_of_the_square_case():
+    # bottom-right alignment: Nq queries against Nk keys are the last Nq rows of
+    # the square causal problem whose queries end with them
+    nk, nq = 40, 13
+    q, k, v = rand(2, 2, nk, 8), rand(2, 2, nk, 8), rand(2, 2, nk, 8)
+    o_sq, l_sq = orc.attention_fwd_ref(q, k, v, 0.3, True)
+    o, lse = orc.attention_fwd_ref(q[:, :, nk - nq :], k, v, 0.3, True)
+    assert np.allclose(o, o_sq[:, :, nk - nq :], atol=1e-14)
+    assert np.allclose(lse, l_sq[:, :, nk - nq :], atol=1e-14)
+
+
+def test_more_queries_than_keys_mask_the_first_rows():
+    nq, nk = 30, 11
+    q, k, v = rand(1, 2, nq, 8), rand(1, 2, nk, 8), rand(1, 2, nk, 8)
+    o, lse = orc.attention_fwd_ref(q, k, v, 0.4, True)
+    assert np.all(o[:, :, : nq - nk] == 0.0) and np.all(np.isneginf(lse[:, :, : nq - nk]))
+    o_sq, l_sq = orc.attention_fwd_ref(q[:, :, nq - nk :], k, v, 0.4, True)
+    assert np.allclose(o[:, :, nq - nk :], o_sq, atol=1e-14)
+    assert np.allclose(lse[:, :, nq - nk :], l_sq, atol=1e-14)
+
+
+def test_single_query_sees_every_key():
+    q, k, v = rand(1, 3, 1, 16), rand(1, 3, 77, 16), rand(1, 3, 77, 16)
+    o_c, l_c = orc.attention_fwd_ref(q, k, v, 0.25, True)
+    o_n, l_n = orc.attention_fwd_ref(q, k, v, 0.25, False)
+    assert np.allclose(o_c, o_n, atol=1e-15) and np.allclose(l_c, l_n, atol=1e-15)
+
+
+def test_unequal_lengths_library_sdpa_cross_check():
+    # torch's SDPA with an explicit boolean mask of the same convention
+    for nq, nk in [(20, 50), (50, 20)]:
+        q, k, v = rand(1, 2, nq, 16), rand(1, 2, nk, 16), rand(1, 2, nk, 16)
+        o, _ = orc.attention_fwd_ref(q, k, v, 0.25, True)
+        keep = torch.ones(nq, nk, dtype=torch.bool).tril(nk - nq)
+        ot = torch.nn.functional.scaled_dot_product_attention(
+            *(torch.from_numpy(x) for x in (q, k, v)), attn_mask=keep, scale=0.25)
+        rows = slice(max(0, nq - nk), nq)  # torch gives NaN on rows with no visible key
+        assert np.allclose(o[:, :, rows], ot.numpy()[:, :, rows], atol=1e-13)
+
+
+@pytest.mark.parametrize("nq,nk", [(200, 300), (300, 200), (130, 500)])
+def test_unequal_lengths_online_loop_and_sampled_rows(nq, nk):
+    q, k, v = rand(1, 2, nq, 8, scale=2.0), rand(1, 2, nk, 8, scale=2.0), rand(1, 2, nk, 8)
+    o1, l1 = orc.attention_fwd_ref(q, k, v, 0.3, True)
+    o2, l2 = orc.online_softmax_attention(q, k, v, 0.3, True, 128, 64)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(l1, l2, atol=1e-12)
+    rows = [np.array([0, 1, nq // 2, nq - 1])] * 2
+    orow, lrow = orc.attention_rows_ref(q, k, v, rows, 0.3, True)
+    for h in range(2):
+        assert np.allclose(orow[0, h], o1[0, h, rows[h]], atol=1e-13)
+        assert np.array_equal(np.isneginf(lrow[0, h]), np.isneginf(l1[0, h, rows[h]]))
+        fin = np.isfinite(l1[0, h, rows[h]])
+        assert np.allclose(lrow[0, h][fin], l1[0, h, rows[h]][fin], atol=1e-13)
+
+
+@pytest.mark.parametrize("nq,nk", [(3, 6), (6, 3)])
+def test_unequal_lengths_backward_finite_differences(nq, nk):
+    d, sc, hh = 3, 0.8, 1e-6
+    q, k, v, do = rand(1, 1, nq, d), rand(1, 1, nk, d), rand(1, 1, nk, d), rand(1, 1, nq, d)
+    dq, dk, dv = orc.attention_bwd_ref(q, k, v, do, sc, True)
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += hh
+            xm[idx] -= hh
+            args = {"q": q, "k": k, "v": v}
+            args[name] = xp
+            lp = _loss(args["q"], args["k"], args["v"], do, sc, True)
+            args[name] = xm
+            lm = _loss(args["q"], args["k"], args["v"], do, sc, True)
+            num[idx] = (lp - lm) / (2 * hh)
+        assert np.linalg.norm(num - g) <= 1e-6 * max(1.0, np.linalg.norm(g)), name
+    if nq > nk:  # queries with no visible key have no gradient
+        assert np.all(dq[:, :, : nq - nk] == 0.0)
+
+
+def test_planted_top_left_alignment_is_caught():
+    # a mask aligned at the top left (j <= i) instead of the bottom right fails the
+    # suffix pin above whenever Nq != Nk
+    nk, nq = 40, 13
+    q, k, v = rand(1, 1, nk, 8), rand(1, 1, nk, 8), rand(1, 1, nk, 8)
+    o_sq, _ = orc.attention_fwd_ref(q, k, v, 0.3, True)
+    s = 0.3 * np.einsum("bhid,bhjd->bhij", q[:, :, nk - nq :], k)
+    s = np.where(np.triu(np.ones((nq, nk), bool), k=1), -np.inf, s)
+    p = orc.safe_softmax(s)
+    o_bad = np.einsum("bhij,bhjd->bhid", p, v)
+    assert not np.allclose(o_bad, o_sq[:, :, nk - nq :], atol=1e-3)
