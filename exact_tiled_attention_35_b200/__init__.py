@@ -17,7 +17,8 @@ import os
 
 import torch
 
-__all__ = ["forward", "backward", "forward_gqa", "backward_gqa", "backward_noalloc", "FAError", "library_path", "load_library", "check_device_status",
+__all__ = ["forward", "backward", "forward_gqa", "backward_gqa", "forward_qk", "backward_qk",
+           "backward_noalloc", "FAError", "library_path", "load_library", "check_device_status",
            "workspace_size", "SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -28,10 +29,12 @@ _P, _I, _F, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 SYMBOLS = {
     "fa_forward": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_forward_gqa": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_forward_qk": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_forward_fp32": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_workspace_size": (_Z, [_I, _I, _I, _I]),
     "fa_backward": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_gqa": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_backward_qk": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_fp32": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_noalloc": (_I, [_P] * 9 + [_I, _I, _I, _I, _F, _I, _P]),
     "fa_debug_wait_timeout": (_I, [_P]),
@@ -164,6 +167,46 @@ def backward_gqa(q, k, v, o, do, lse, causal=False, scale=None, workspace=None):
                                _ptr(dk), _ptr(dv), _ptr(workspace),
                                workspace.numel() * workspace.element_size(), B, H, Hkv, N, d, scale,
                                int(bool(causal)), _stream(q)), "fa_backward_gqa")
+    return dq, dk, dv
+
+
+def forward_qk(q, k, v, causal=False, scale=None, out=None, lse=None):
+    """Forward with separate query and key lengths via fa_forward_qk (bf16).
+
+    q: [B, H, Nq, d]; k, v: [B, Hkv, Nk, d] with Hkv dividing H.  The causal
+    mask is aligned at the bottom right (key j visible to query i iff
+    j <= i + Nk - Nq); a query that sees no key gets O = 0 and LSE = -inf."""
+    B, H, Nq, d = _shape(q)
+    Hkv, Nk = int(k.shape[1]), int(k.shape[2])
+    _require((q,), torch.bfloat16, (B, H, Nq, d))
+    _require((k, v), torch.bfloat16, (B, Hkv, Nk, d))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _require((out,), torch.bfloat16, (B, H, Nq, d))
+    _require((lse,), torch.float32, (B, H, Nq))
+    _check(load_library().fa_forward_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Hkv, Nq,
+                                        Nk, d, scale, int(bool(causal)), _stream(q)), "fa_forward_qk")
+    return out, lse
+
+
+def backward_qk(q, k, v, o, do, lse, causal=False, scale=None, workspace=None):
+    """dQ [B,H,Nq,d], dK and dV [B,Hkv,Nk,d] via fa_backward_qk (bf16)."""
+    B, H, Nq, d = _shape(q)
+    Hkv, Nk = int(k.shape[1]), int(k.shape[2])
+    _require((q, o, do), torch.bfloat16, (B, H, Nq, d))
+    _require((k, v), torch.bfloat16, (B, Hkv, Nk, d))
+    _require((lse,), torch.float32, (B, H, Nq))
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    lib = load_library()
+    if workspace is None:
+        workspace = torch.empty(max(int(lib.fa_backward_workspace_size(B, H, Nq, d)), 16),
+                                dtype=torch.uint8, device=q.device)
+    _check(lib.fa_backward_qk(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                              _ptr(dk), _ptr(dv), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), B, H, Hkv, Nq, Nk, d, scale,
+                              int(bool(causal)), _stream(q)), "fa_backward_qk")
     return dq, dk, dv
 
 

@@ -127,32 +127,34 @@ namespace fa {
 namespace {
 
 fa_status forward_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                       int H, int Hkv, int N, int d, float scale, int causal, void* stream) {
-  fa_status s = check_shape(B, H, N, d, scale);
+                       int H, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                       void* stream) {
+  fa_status s = check_shape(B, H, Nq, d, scale);
   if (s != FA_OK) return s;
+  if ((s = check_shape(B, H, Nk, d, scale)) != FA_OK) return s;
   if (Hkv <= 0 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if ((s = check_ptrs({q, k, v, o, lse})) != FA_OK) return s;
   if ((s = check_device()) != FA_OK) return s;
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, d, N, B * H) || !make_map(&mk, k, d, N, B * Hkv) ||
-      !make_map(&mv, v, d, N, B * Hkv))
+  if (!make_map(&mq, q, d, Nq, B * H) || !make_map(&mk, k, d, Nk, B * Hkv) ||
+      !make_map(&mv, v, d, Nk, B * Hkv))
     return map_failed();
-  return from_cuda(sm100_forward(mq, mk, mv, o, lse, B, H, Hkv, N, d, scale, causal ? 1 : 0,
+  return from_cuda(sm100_forward(mq, mk, mv, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal ? 1 : 0,
                                  static_cast<cudaStream_t>(stream)));
 }
 
 fa_status backward_bf16(const void* q, const void* k, const void* v, const void* o,
                         const void* dout, const float* lse, void* dq, void* dk, void* dv,
-                        void* workspace, int B, int H, int Hkv, int N, int d, float scale,
-                        int causal, void* stream) {
+                        void* workspace, int B, int H, int Hkv, int Nq, int Nk, int d,
+                        float scale, int causal, void* stream) {
   const int BH = B * H;
   CUtensorMap mq, mk, mv, mdo, mdq;
-  if (!make_map(&mq, q, d, N, BH) || !make_map(&mk, k, d, N, B * Hkv) ||
-      !make_map(&mv, v, d, N, B * Hkv) || !make_map(&mdo, dout, d, N, BH) ||
-      !make_dq_map(&mdq, static_cast<char*>(workspace) + sm100_backward_dq_offset(BH, N), d, N, BH))
+  if (!make_map(&mq, q, d, Nq, BH) || !make_map(&mk, k, d, Nk, B * Hkv) ||
+      !make_map(&mv, v, d, Nk, B * Hkv) || !make_map(&mdo, dout, d, Nq, BH) ||
+      !make_dq_map(&mdq, static_cast<char*>(workspace) + sm100_backward_dq_offset(BH, Nq), d, Nq, BH))
     return map_failed();
   return from_cuda(sm100_backward(mq, mk, mv, mdo, mdq, o, dout, lse, dq, dk, dv, workspace, B, H,
-                                  Hkv, N, d, scale, causal ? 1 : 0,
+                                  Hkv, Nq, Nk, d, scale, causal ? 1 : 0,
                                   static_cast<cudaStream_t>(stream)));
 }
 
@@ -178,12 +180,18 @@ extern "C" {
 
 fa_status fa_forward(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                      int N, int d, float scale, int causal, void* stream) {
-  return forward_bf16(q, k, v, o, lse, B, H, H, N, d, scale, causal, stream);
+  return forward_bf16(q, k, v, o, lse, B, H, H, N, N, d, scale, causal, stream);
 }
 
 fa_status fa_forward_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                          int H, int Hkv, int N, int d, float scale, int causal, void* stream) {
-  return forward_bf16(q, k, v, o, lse, B, H, Hkv, N, d, scale, causal, stream);
+  return forward_bf16(q, k, v, o, lse, B, H, Hkv, N, N, d, scale, causal, stream);
+}
+
+fa_status fa_forward_qk(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int H, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                        void* stream) {
+  return forward_bf16(q, k, v, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal, stream);
 }
 
 fa_status fa_forward_fp32(const float* q, const float* k, const float* v, float* o, float* lse, int B,
@@ -210,7 +218,7 @@ fa_status fa_backward(const void* q, const void* k, const void* v, const void* o
   if (workspace == nullptr || ws_bytes < ws_bytes_for(B, H, N, d)) return FA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
   if ((s = check_device()) != FA_OK) return s;
-  return backward_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, H, N, d, scale, causal,
+  return backward_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, H, N, N, d, scale, causal,
                        stream);
 }
 
@@ -225,8 +233,24 @@ fa_status fa_backward_gqa(const void* q, const void* k, const void* v, const voi
   if (workspace == nullptr || ws_bytes < ws_bytes_for(B, H, N, d)) return FA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
   if ((s = check_device()) != FA_OK) return s;
-  return backward_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, d, scale, causal,
+  return backward_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, N, N, d, scale, causal,
                        stream);
+}
+
+fa_status fa_backward_qk(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                         void* workspace, size_t ws_bytes, int B, int H, int Hkv, int Nq, int Nk,
+                         int d, float scale, int causal, void* stream) {
+  fa_status s = check_shape(B, H, Nq, d, scale);
+  if (s != FA_OK) return s;
+  if ((s = check_shape(B, H, Nk, d, scale)) != FA_OK) return s;
+  if (Hkv <= 0 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv})) != FA_OK) return s;
+  if (workspace == nullptr || ws_bytes < ws_bytes_for(B, H, Nq, d)) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
+  if ((s = check_device()) != FA_OK) return s;
+  return backward_bf16(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, Nq, Nk, d, scale,
+                       causal, stream);
 }
 
 fa_status fa_backward_fp32(const float* q, const float* k, const float* v, const float* o,
@@ -320,6 +344,6 @@ extern "C" fa_status fa_backward_noalloc(const void* q, const void* k, const voi
   if ((s = check_device()) != FA_OK) return s;
   void* scratch = noalloc_scratch();
   if (scratch == nullptr) return FA_ERR_CUDA;
-  return backward_bf16(q, k, v, o, dout, lse, dq, dk, dv, scratch, B, H, H, N, d, scale, causal,
+  return backward_bf16(q, k, v, o, dout, lse, dq, dk, dv, scratch, B, H, H, N, N, d, scale, causal,
                        stream);
 }

@@ -90,9 +90,12 @@ struct Params {
   int BHkv;    // key/value heads B*Hkv
   int H;       // query heads per batch
   int G;       // query heads per key/value head (H / Hkv; 1 without grouping)
-  int N;
-  int Npad;
-  int nkv;             // number of key tiles = Npad / 128
+  int Nq;              // query rows
+  int Nk;              // key rows
+  int off;             // Nk - Nq: under the causal mask key j is visible to query i iff j <= i + off
+  int Npad;            // Nq rounded up to whole 128-row tiles (the LSE / D vectors)
+  int nq;              // number of query tiles = Npad / 128
+  int nkv;             // number of key tiles
   int chunk;           // key/value heads per locality chunk
   float scale;
   float scale_log2;
@@ -186,8 +189,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   const int h0 = chunk_id * p.chunk, hn = min(p.chunk, p.BHkv - h0);
   const int j = w_in / hn;
   const int bkv = h0 + (w_in - j * hn);  // key/value head
-  const int nq = p.nkv;
-  const int i0 = p.causal ? j : 0;
+  const int nq = p.nq;
+  // first query tile with a row that sees a key of tile j (the causal mask is
+  // aligned bottom right: key k visible to query r iff k <= r + off)
+  const int i0 = p.causal ? max(0, j * BN - p.off) / BM : 0;
   const int nqi = nq - i0;        // query tiles per query head
   const int niter = p.G * nqi;    // every query head of the group, then its query tiles
   // query head and query tile of iteration it
@@ -380,7 +385,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int qw = warp % 4, h = warp / 4;
     const int r = qw * 32 + lane;
     const int kr = j * BN + r;
-    const bool key_ok = kr < p.N;
+    const bool key_ok = kr < p.Nk;
     const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::T_S;
     const uint32_t tDP = tmem + lane_off + C::T_DP;
@@ -405,7 +410,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int e = 0; e < 32; ++e) pr[cc * 32 + e] = __uint_as_float(v[e]);
       }
       tmem_wait_ld();
-      const bool diag = p.causal && i == j;
+      // Masked keys get S = -inf before the exponentials (P = 0): key j*BN + r is
+      // hidden from query i*BM + 64h + col iff col < hide (above the causal
+      // diagonal), and from every query if it is past Nk.
+      {
+        const int hide = !key_ok ? 64 : p.causal ? min(max(r + (j - i) * BN - p.off - h * 64, 0), 64) : 0;
+        if (hide > 0) {
+#pragma unroll
+          for (int col = 0; col < 64; ++col)
+            if (col < hide) pr[col] = -INFINITY;
+        }
+      }
       const uint64_t c2 = f2_pack(c, c);
 #pragma unroll
       for (int c4 = 0; c4 < 16; ++c4) {
@@ -418,11 +433,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         pr[4 * c4 + 1] = ex2(x1);
         pr[4 * c4 + 2] = ex2(x2);
         pr[4 * c4 + 3] = ex2(x3);
-      }
-      if (!key_ok || diag) {  // masked keys: rows past N, and keys above the diagonal
-#pragma unroll
-        for (int col = 0; col < 64; ++col)
-          if (!key_ok || h * 64 + col < r) pr[col] = 0.f;
       }
       {
         uint32_t v[32];
@@ -474,7 +484,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (ok) ok = mbar_wait(&bars->all_done, 0, 44);
     if (ok) {
       tc_fence_after();
-      const size_t row = (size_t)bkv * p.N + (size_t)(key_ok ? kr : 0);
+      const size_t row = (size_t)bkv * p.Nk + (size_t)(key_ok ? kr : 0);
 #pragma unroll
       for (int which = 0; which < 2; ++which) {
         const uint32_t tsrc = tmem + lane_off + (which ? C::T_DV : C::T_DK) + h * DH;
@@ -536,7 +546,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         __syncwarp();
         if (lane == 0) {
           // rows past N are clipped by the tensor map; a box wholly past N is skipped
-          if (row0 < p.N) tma_reduce_add_3d(&mdq, buf, cc * 32, row0, bh);
+          if (row0 < p.Nq) tma_reduce_add_3d(&mdq, buf, cc * 32, row0, bh);
           asm volatile("cp.async.bulk.commit_group;" ::: "memory");
         }
       }
@@ -589,7 +599,9 @@ __global__ void __launch_bounds__(256) preprocess_kernel(const __nv_bfloat16* __
   for (int c = lane; c < D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (lane == 0) {
     dsum[gw] = -acc;
-    lse2[gw] = -lse[(size_t)bh * N + row] * kLog2e;
+    // a row that saw no key in the forward (LSE = -inf) gets probability 0 too
+    const float l = lse[(size_t)bh * N + row];
+    lse2[gw] = l == -INFINITY ? -INFINITY : -l * kLog2e;
   }
 }
 
@@ -607,13 +619,13 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict
 }
 
 // Key/value heads per locality chunk.  Per key/value head the pass touches
-// K and V (4 N d bytes), the Q and dO of its G query heads (4 G N d bytes) and
-// their fp32 dQ accumulator (4 G N d bytes), which the reduce-adds must find in
+// K and V (4 Nk d bytes), the Q and dO of its G query heads (4 G Nq d bytes) and
+// their fp32 dQ accumulator (4 G Nq d bytes), which the reduce-adds must find in
 // L2; a chunk keeps that near 80 MB of the 126 MB L2.  A chunk also holds at
 // least two waves of CTAs so that its light tail balances the SMs, and chunks
 // split the heads evenly.
-inline int chunk_heads(int BHkv, int G, int N, int d, int nkv, int sms) {
-  const long long per_head = 4LL * N * d * (2LL * G + 1);
+inline int chunk_heads(int BHkv, int G, int Nq, int Nk, int d, int nkv, int sms) {
+  const long long per_head = 4LL * d * (Nk + 2LL * G * Nq);
   long long c = std::max(1LL, (80LL << 20) / per_head);
   c = std::max<long long>(c, (2LL * sms + nkv - 1) / nkv);
   c = std::min<long long>(c, BHkv);
@@ -639,8 +651,9 @@ cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const C
                            const CUtensorMap& mdo, const CUtensorMap& mdq, const void* o,
                            const void* dout, const float* lse,
                            void* dq, void* dk, void* dv, void* workspace, int B, int H, int Hkv,
-                           int N, int d, float scale, int causal, cudaStream_t st) {
+                           int Nq, int Nk, int d, float scale, int causal, cudaStream_t st) {
   const int BH = B * H;
+  const int N = Nq;  // the workspace and the preprocess run over query rows
   const int npad = (N + 127) / 128 * 128;
   const size_t vec = ((size_t)BH * npad * 4 + 255) / 256 * 256;
   float* lse2 = static_cast<float*>(workspace);
@@ -667,16 +680,19 @@ cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const C
   p.BHkv = B * Hkv;
   p.H = H;
   p.G = H / Hkv;
-  p.N = N;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.off = Nk - Nq;
   p.Npad = npad;
-  p.nkv = npad / 128;
+  p.nq = npad / 128;
+  p.nkv = (Nk + 127) / 128;
   p.scale = scale;
   p.scale_log2 = scale * bwd::kLog2e;
   p.causal = causal;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  p.chunk = bwd::chunk_heads(p.BHkv, p.G, N, d, p.nkv, std::max(sms, 1));
+  p.chunk = bwd::chunk_heads(p.BHkv, p.G, Nq, Nk, d, p.nkv, std::max(sms, 1));
   const dim3 grid((unsigned)(p.nkv * p.BHkv));
   if (d == 128) {
     const int smem = bwd::Cfg<128>::SMEM_BYTES;

@@ -84,8 +84,10 @@ struct Params {
   int BH;      // query heads B*H
   int H;       // query heads per batch
   int G;       // query heads per key/value head (1 without grouping)
-  int N;
-  int npairs;  // ceil(N / 256)
+  int Nq;      // query rows
+  int Nk;      // key rows
+  int off;     // Nk - Nq: under the causal mask key j is visible to query i iff j <= i + off
+  int npairs;  // ceil(Nq / 256)
   int chunk;   // query heads per locality chunk (their K/V stay resident in L2)
   int items;   // work items = query-tile pairs x heads
   int slot;    // ticket counter of this launch
@@ -118,12 +120,15 @@ struct Bars {
 // issued in between.
 __device__ unsigned int g_fwd_tickets[kSchedSlots][2];
 
-// number of key tiles query tile starting at row q0 needs (0 if the tile is empty)
-__device__ __forceinline__ int tiles_for(int q0, int N, int causal) {
-  if (q0 >= N) return 0;
-  const int nkv = (N + BN - 1) / BN;
-  if (!causal) return nkv;
-  return min(nkv, q0 / BN + 1);
+// Number of key tiles the query tile starting at row q0 needs: 0 past the last
+// query, and 0 too when the causal mask hides every key from every row of the
+// tile (possible when Nq > Nk; those rows get O = 0 and LSE = -inf).
+__device__ __forceinline__ int tiles_for(int q0, const Params& p) {
+  if (q0 >= p.Nq) return 0;
+  const int nkv = (p.Nk + BN - 1) / BN;
+  if (!p.causal) return nkv;
+  const int kmax = min(q0 + BM - 1, p.Nq - 1) + p.off;  // last key the tile's last row sees
+  return kmax < 0 ? 0 : min(nkv, kmax / BN + 1);
 }
 
 // Work item -> (query head, query-tile pair).  The heads are cut into chunks
@@ -165,7 +170,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     it.bkv = (it.bh / p.H) * (p.H / p.G) + (it.bh % p.H) / p.G;
     it.qbase = pair * (NQT * BM);
 #pragma unroll
-    for (int t = 0; t < NQT; ++t) it.n[t] = tiles_for(it.qbase + t * BM, p.N, p.causal);
+    for (int t = 0; t < NQT; ++t) it.n[t] = tiles_for(it.qbase + t * BM, p);
     it.nmax = max(it.n[0], it.n[1]);
     return it;
   };
@@ -322,6 +327,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (ok) mbar_arrive(&bars->it_empty[r % kItemRing]);
         if (!ok || item >= p.items) break;
         const Item w = item_info(item);
+        if (w.nmax == 0) continue;  // every key hidden from both tiles: nothing to multiply
         for (int t = 0; t < NQT && ok; ++t)
           if (w.n[t] > 0) ok = mbar_wait(&bars->q_full[t], qcnt[t] & 1, 3);
         if (ok) ok = mbar_wait(&bars->kv_full[kslot], kphase, 4);
@@ -405,9 +411,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (!ok || item >= p.items) break;
     const Item w = item_info(item);
     const int n = w.n[t];
-    if (n == 0) continue;
     const int bh = w.bh;
     const int q_row = w.qbase + t * BM + row;
+    if (n == 0) {
+      // no key visible to any row of this tile (or no tile): O = 0, LSE = -inf
+      if (q_row < p.Nq) {
+        uint4* orow = reinterpret_cast<uint4*>(p.o + ((size_t)bh * p.Nq + q_row) * D);
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) orow[i] = make_uint4(0u, 0u, 0u, 0u);
+        p.lse[(size_t)bh * p.Nq + q_row] = -INFINITY;
+      }
+      continue;
+    }
+    const int q_tile0 = w.qbase + t * BM;
     float m_used = -INFINITY, l = 0.f;
     for (int j = 0; j < n && ok; ++j) {
       ok = mbar_wait(&bars->s_full[t], (gtile + j) & 1, 16 + t);
@@ -423,9 +439,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       tmem_wait_ld();
       const int k0 = j * BN;
-      const bool need_mask = (p.causal && j == n - 1) || (k0 + BN > p.N);
+      // masked keys in this tile: past Nk, or above the causal diagonal of some row
+      const bool need_mask = (p.causal && k0 + BN - 1 > q_tile0 + p.off) || (k0 + BN > p.Nk);
       if (need_mask) {
-        const int lim = p.causal ? min(q_row + 1, p.N) : p.N;  // keys < lim are visible
+        const int lim = p.causal ? min(q_row + 1 + p.off, p.Nk) : p.Nk;  // keys < lim are visible
 #pragma unroll
         for (int i = 0; i < BN; ++i)
           if (k0 + i >= lim) s[i] = -INFINITY;
@@ -485,13 +502,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (ok) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = p.o + ((size_t)bh * p.N + (size_t)(q_row < p.N ? q_row : 0)) * D;
+      __nv_bfloat16* orow = p.o + ((size_t)bh * p.Nq + (size_t)(q_row < p.Nq ? q_row : 0)) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t r[32];
         tmem_ld32(tO + cc * 32, r);
         tmem_wait_ld();
-        if (q_row < p.N) {
+        if (q_row < p.Nq) {
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i)
@@ -501,8 +518,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
-      if (q_row < p.N)
-        p.lse[(size_t)bh * p.N + q_row] = l > 0.f ? m_used * p.scale + logf(l) : -INFINITY;
+      if (q_row < p.Nq)
+        p.lse[(size_t)bh * p.Nq + q_row] = l > 0.f ? m_used * p.scale + logf(l) : -INFINITY;
     }
     gtile += n;
     ++icnt;
@@ -536,8 +553,8 @@ inline int chunk_heads(int BH, int G, int N, int d, int npairs, int grid) {
 }  // namespace fwd
 
 cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                          void* o, float* lse, int B, int H, int Hkv, int N, int d, float scale,
-                          int causal, cudaStream_t st) {
+                          void* o, float* lse, int B, int H, int Hkv, int Nq, int Nk, int d,
+                          float scale, int causal, cudaStream_t st) {
   const int BH = B * H;
   fwd::Params p;
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -545,8 +562,10 @@ cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   p.BH = BH;
   p.H = H;
   p.G = H / Hkv;
-  p.N = N;
-  p.npairs = (N + 2 * fwd::BM - 1) / (2 * fwd::BM);
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.off = Nk - Nq;
+  p.npairs = (Nq + 2 * fwd::BM - 1) / (2 * fwd::BM);
   p.scale = scale;
   p.scale_log2 = scale * fwd::kLog2e;
   p.causal = causal;
@@ -556,7 +575,7 @@ cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const dim3 grid((unsigned)std::min(p.items, std::max(sms, 1)));
-  p.chunk = fwd::chunk_heads(BH, p.G, N, d, p.npairs, (int)grid.x);
+  p.chunk = fwd::chunk_heads(BH, p.G, Nk, d, p.npairs, (int)grid.x);
   static std::atomic<unsigned int> launches{0};
   p.slot = (int)(launches.fetch_add(1u, std::memory_order_relaxed) % fwd::kSchedSlots);
   cudaError_t e;

@@ -16,22 +16,26 @@ cudaError_t simt_backward(bool bf16, const void* q, const void* k, const void* v
                           int N, int d, float scale, int causal, cudaStream_t st);
 
 // tcgen05 forward (fa_fwd_sm100.cu).  Tensor maps: 3-D bf16 views
-// {d, N, heads} of Q (B*H heads), K and V (B*Hkv heads) with a {64, 128, 1} box
-// and 128-byte swizzle.  Hkv divides H (Hkv = H: plain multi-head attention).
+// {d, Nq, heads} of Q (B*H heads) and {d, Nk, heads} of K and V (B*Hkv heads)
+// with a {64, 128, 1} box and 128-byte swizzle.  Hkv divides H (Hkv = H: plain
+// multi-head attention).  Under the causal mask key j is visible to query i iff
+// j <= i + Nk - Nq.
 cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                          void* o, float* lse, int B, int H, int Hkv, int N, int d, float scale,
-                          int causal, cudaStream_t st);
+                          void* o, float* lse, int B, int H, int Hkv, int Nq, int Nk, int d,
+                          float scale, int causal, cudaStream_t st);
 
 // tcgen05 backward (fa_bwd_sm100.cu): preprocess, main and dQ-convert kernels.
-// Workspace layout: LSE*log2(e) [BH, Npad], D [BH, Npad], fp32 dQ [BH, N, d].
+// Workspace layout (N = query rows): LSE*log2(e) [BH, Npad], D [BH, Npad],
+// fp32 dQ [BH, N, d].
 size_t sm100_backward_workspace(int BH, int N, int d);
 // byte offset of the fp32 dQ accumulator inside the workspace
 size_t sm100_backward_dq_offset(int BH, int N);
-// mdq: 3-D fp32 view {d, N, B*H} of the accumulator, box {32, 32, 1}, 128-byte swizzle
+// mq, mdo, mdq over Nq rows; mk, mv over Nk rows.
+// mdq: 3-D fp32 view {d, Nq, B*H} of the accumulator, box {32, 32, 1}, 128-byte swizzle
 cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                            const CUtensorMap& mdo, const CUtensorMap& mdq, const void* o,
                            const void* dout, const float* lse,
                            void* dq, void* dk, void* dv, void* workspace, int B, int H, int Hkv,
-                           int N, int d, float scale, int causal, cudaStream_t st);
+                           int Nq, int Nk, int d, float scale, int causal, cudaStream_t st);
 
 }  // namespace fa

@@ -69,6 +69,18 @@ fa_status fa_forward_gqa(const void* q, const void* k, const void* v, void* o, f
                          int B, int H, int Hkv, int N, int d, float scale, int causal,
                          void* stream);
 
+/* Forward pass with separate query and key lengths (bf16, grouped-query heads
+ * as in fa_forward_gqa).  q, o: [B,H,Nq,d]; k, v: [B,Hkv,Nk,d]; lse: fp32
+ * [B,H,Nq].  Nq = Nk is fa_forward_gqa.  Under the causal mask, which the pages
+ * define only for square attention, the mask is aligned at the bottom right:
+ * key j is visible to query i iff j <= i + (Nk - Nq), so the last query sees
+ * every key (the suffix of a longer square problem, e.g. new queries against
+ * a key/value cache).  A query that sees no key (i < Nq - Nk) gets O = 0 and
+ * LSE = -inf.  Errors as for fa_forward; Nq and Nk must both be >= 1. */
+fa_status fa_forward_qk(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int H, int Hkv, int Nq, int Nk, int d, float scale, int causal,
+                        void* stream);
+
 /* Forward pass with fp32 storage (q, k, v, o are float [B,H,N,d]); fp32
  * arithmetic on CUDA cores.  Same definition, same LSE convention. */
 fa_status fa_forward_fp32(const float* q, const float* k, const float* v, float* o, float* lse,
@@ -100,6 +112,15 @@ fa_status fa_backward_gqa(const void* q, const void* k, const void* v, const voi
                           const void* dout, const float* lse, void* dq, void* dk, void* dv,
                           void* workspace, size_t ws_bytes, int B, int H, int Hkv, int N, int d,
                           float scale, int causal, void* stream);
+
+/* Backward pass of fa_forward_qk: q, o, dout, dq: [B,H,Nq,d]; k, v, dk, dv:
+ * [B,Hkv,Nk,d]; lse: [B,H,Nq] as written by fa_forward_qk (rows with LSE = -inf
+ * have P = 0 and contribute nothing).  Workspace:
+ * fa_backward_workspace_size(B, H, Nq, d), i.e. sized by the query rows. */
+fa_status fa_backward_qk(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                         void* workspace, size_t ws_bytes, int B, int H, int Hkv, int Nq, int Nk,
+                         int d, float scale, int causal, void* stream);
 
 /* Backward pass with fp32 storage (all tensors float); CUDA-core arithmetic.
  * Workspace as for fa_backward. */

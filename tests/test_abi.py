@@ -99,3 +99,28 @@ def test_backward_rejects_bad_arguments(lib, fn):
         bad[i] = None
         assert f(*bad, ws, need, 1, 2, 300, 64, 0.125, 0, None) == INVALID
     assert f(*ptrs, ws, need, 1, 2, 300, 80, 0.125, 0, None) == UNSUPPORTED
+
+
+def test_unequal_length_entry_points_reject_bad_arguments(lib):
+    # host-side checks only: no CUDA call is reached
+    f = lib.fa_forward_qk
+    assert f(*GOOD, 1, 4, 2, 0, 128, 64, 0.125, 1, None) == INVALID  # Nq = 0
+    assert f(*GOOD, 1, 4, 2, 128, 0, 64, 0.125, 1, None) == INVALID  # Nk = 0
+    assert f(*GOOD, 1, 4, 3, 128, 256, 64, 0.125, 1, None) == INVALID  # Hkv does not divide H
+    assert f(*GOOD, 1, 4, 2, 128, 256, 96, 0.125, 1, None) == UNSUPPORTED
+    for i in range(5):
+        ptrs = list(GOOD)
+        ptrs[i] = None
+        assert f(*ptrs, 1, 4, 2, 100, 300, 64, 0.125, 1, None) == INVALID
+    b = lib.fa_backward_qk
+    ptrs = [P(0x10000 * (i + 1)) for i in range(9)]
+    ws = P(0x100000)
+    need = lib.fa_backward_workspace_size(1, 4, 100, 64)  # sized by the query rows
+    assert b(*ptrs, ws, need - 1, 1, 4, 2, 100, 300, 64, 0.125, 1, None) == WORKSPACE
+    assert b(*ptrs, P(0x100004), need, 1, 4, 2, 100, 300, 64, 0.125, 1, None) == MISALIGNED
+    assert b(*ptrs, ws, need, 1, 4, 2, 100, 0, 64, 0.125, 1, None) == INVALID
+    assert b(*ptrs, ws, need, 1, 4, 2, 0, 300, 64, 0.125, 1, None) == INVALID
+    for i in range(9):
+        bad = list(ptrs)
+        bad[i] = None
+        assert b(*bad, ws, need, 1, 4, 2, 100, 300, 64, 0.125, 1, None) == INVALID

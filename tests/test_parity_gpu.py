@@ -289,3 +289,74 @@ def test_gqa_with_full_heads_matches_multi_head_bitwise():
     o1, l1 = fa.forward(q, k, v, causal=True)
     o2, l2 = fa.forward_gqa(q, k, v, causal=True)
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# ---------------------------------------------------------------- unequal query / key lengths
+
+
+def _check_fwd_with_empty_rows(o, lse, o_ref, lse_ref, what):
+    # rows that see no key: O = 0 and LSE = -inf exactly; the rest as check_fwd
+    empty = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lse), empty), what
+    assert np.all(o[empty] == 0.0), what
+    full = ~empty
+    if np.any(full):
+        check_fwd(o[full], lse[full], o_ref[full], lse_ref[full], what)
+
+
+def _qk_inputs(B, H, Hkv, Nq, Nk, d, seed):
+    q, do = make_inputs(B, H, Nq, d, seed=seed, with_do=True)[0::3]
+    k, v = make_inputs(B, Hkv, Nk, d, seed=seed + 100)[1:3]
+    return q, k, v, do
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Nq,Nk", [(1, 1000), (77, 300), (128, 1024), (300, 77), (1000, 1), (384, 130),
+                                   (200, 201), (640, 256)])
+def test_forward_unequal_lengths(Nq, Nk, causal, d):
+    from oracle import attention_fwd_gqa_ref
+
+    q, k, v, _ = _qk_inputs(1, 4, 2, Nq, Nk, d, seed=Nq + Nk)
+    o, lse = fa.forward_qk(*(t.cuda() for t in (q, k, v)), causal=causal)
+    fa.check_device_status()
+    o_ref, lse_ref = attention_fwd_gqa_ref(to_f64(q), to_f64(k), to_f64(v), 1 / math.sqrt(d), causal)
+    _check_fwd_with_empty_rows(to_f64(o), to_f64(lse), o_ref, lse_ref, (Nq, Nk, causal, d))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Nq,Nk", [(77, 300), (300, 77), (128, 640), (1, 200), (200, 1), (250, 384)])
+def test_backward_unequal_lengths(Nq, Nk, causal, d):
+    from oracle import attention_bwd_gqa_ref
+
+    q, k, v, do = _qk_inputs(1, 4, 2, Nq, Nk, d, seed=7 * Nq + Nk)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = fa.forward_qk(qd, kd, vd, causal=causal)
+    dq, dk, dv = fa.backward_qk(qd, kd, vd, o, dod, lse, causal=causal)
+    fa.check_device_status()
+    ref = attention_bwd_gqa_ref(to_f64(q), to_f64(k), to_f64(v), to_f64(do), 1 / math.sqrt(d), causal)
+    check_bwd(tuple(to_f64(x) for x in (dq, dk, dv)), ref, (Nq, Nk, causal, d))
+
+
+def test_unequal_lengths_equal_to_square_entry_points():
+    q, k, v, do = _qk_inputs(2, 4, 4, 384, 384, 128, seed=5)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o1, l1 = fa.forward_qk(qd, kd, vd, causal=True)
+    o2, l2 = fa.forward(qd, kd, vd, causal=True)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    g1 = fa.backward_qk(qd, kd, vd, o1, dod, l1, causal=True)
+    g2 = fa.backward(qd, kd, vd, o2, dod, l2, causal=True)
+    assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])  # dK, dV: one CTA each
+    assert float((g1[0].float() - g2[0].float()).norm() / g2[0].float().norm()) < 1e-3
+
+
+def test_fewer_queries_are_the_last_rows_of_the_square_case_on_gpu():
+    # bottom-right alignment on the device: new queries against a longer key/value
+    # sequence reproduce the last rows of the square causal problem
+    q, k, v, _ = _qk_inputs(1, 4, 4, 1000, 1000, 128, seed=6)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o_sq, l_sq = fa.forward(qd, kd, vd, causal=True)
+    o, lse = fa.forward_qk(qd[:, :, 1000 - 300 :].contiguous(), kd, vd, causal=True)
+    assert max_abs(to_f64(o), to_f64(o_sq[:, :, 700:])) <= 1e-2
+    assert max_abs(to_f64(lse), to_f64(l_sq[:, :, 700:])) <= 1e-4
