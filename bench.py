@@ -98,15 +98,21 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons for one GPU while running."""
+    """Samples nvidia-smi clocks and throttle reasons for one GPU while running.
 
-    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Rows carry nvidia-smi's timestamp, so the samples of a time window (for
+    example the timed steps and the soak right before them) can be picked out."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, device):
+    def __init__(self, device, interval_ms=50):
         self.proc = None
         self.path = None
+        self.interval_ms = interval_ms
+        self.rows = []
         try:
             self.uuid = str(torch.cuda.get_device_properties(device).uuid)
         except Exception:
@@ -117,7 +123,7 @@ class ClockSampler:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                   "-lms", "100"]
+                   "-lms", str(self.interval_ms)]
             if self.uuid:
                 cmd += ["-i", "GPU-" + self.uuid if not self.uuid.startswith("GPU-") else self.uuid]
             self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
@@ -127,35 +133,42 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is None:
-            return None
+            return
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        rows = []
+        import datetime
+
         with open(self.path) as f:
             for line in f:
                 parts = [x.strip() for x in line.split(",")]
                 if len(parts) < 10:
                     continue
                 try:
-                    rows.append((float(parts[2]), float(parts[3]), float(parts[4]), parts[5:]))
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    self.rows.append((ts, float(parts[2]), float(parts[3]), float(parts[4]), parts[6:10]))
                 except ValueError:
                     continue
         os.unlink(self.path)
+
+    def summary(self, t0=None, t1=None, what=""):
+        """Clock record of the samples taken between host times t0 and t1."""
+        rows = [r for r in self.rows if (t0 is None or r[0] >= t0) and (t1 is None or r[0] <= t1)]
         if not rows:
             return None
         reasons = set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
-            for name, flag in zip(names, r[3][1:]):
+            for name, flag in zip(self.REASONS, r[4]):
                 if flag.lower().startswith("active"):
                     reasons.add(name)
-        loaded = [r for r in rows if r[2] > 300.0] or rows
-        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
-                "power_w_max": max(r[2] for r in rows), "samples": len(rows),
-                "reasons": sorted(reasons)}
+        loaded = [r for r in rows if r[3] > 300.0] or rows
+        return {"sm_mhz": statistics.median(r[1] for r in loaded), "sm_max_mhz": max(r[2] for r in rows),
+                "power_w_max": max(r[3] for r in rows), "samples": len(rows),
+                "samples_under_load": len([r for r in rows if r[3] > 300.0]),
+                "window_s": round(rows[-1][0] - rows[0][0], 3), "reasons": sorted(reasons),
+                "covers": what}
 
 
 # ------------------------------------------------------------ distributed
@@ -252,80 +265,208 @@ def run_reference(args, w, world, rank):
 # ----------------------------------------------------------------- GPU arm
 
 
+def _vp(t):
+    import ctypes
+
+    return ctypes.c_void_p(t.data_ptr())
+
+
+class Problem:
+    """Device buffers of one workload plus pre-marshalled C-ABI argument lists, so
+    the timed loops call the library with no per-call Python checks."""
+
+    def __init__(self, w, dev, seed, lib, stream):
+        import ctypes
+
+        self.w = w
+        ts = make_inputs(w.B, w.H, w.N, w.d, dtype=w.dtype, seed=seed, qk_gain=w.qk_gain,
+                         with_do=w.backward)
+        q, k, v = ts[:3]
+        do = ts[3] if w.backward else None
+        self.host = list(ts)
+        self.q, self.k, self.v = (t.to(dev) for t in (q, k, v))
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+        st = ctypes.c_void_p(stream.cuda_stream)
+        causal = int(w.causal)
+        self.fwd_fn = lib.fa_forward if w.dtype == torch.bfloat16 else lib.fa_forward_fp32
+        if w.backward and w.dtype != torch.bfloat16:
+            raise ValueError("the timed backward runs the bf16 path")
+        self.fwd_args = (_vp(self.q), _vp(self.k), _vp(self.v), _vp(self.o), _vp(self.lse), w.B, w.H, w.N,
+                         w.d, w.scale, causal, st)
+        if w.backward:
+            self.do = do.to(dev)
+            self.dq, self.dk, self.dv = (torch.empty_like(t) for t in (self.q, self.k, self.v))
+            ws_bytes = int(lib.fa_backward_workspace_size(w.B, w.H, w.N, w.d))
+            self.ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+            self.bwd_fn = lib.fa_backward_stages
+            self.bwd_args = [_vp(t) for t in (self.q, self.k, self.v, self.o, self.do, self.lse, self.dq,
+                                               self.dk, self.dv, self.ws)]
+            self.bwd_tail = (self.ws.numel(), w.B, w.H, w.H, w.N, w.N, w.d, w.scale, causal)
+            self.stream = st
+
+    def forward(self):
+        return self.fwd_fn(*self.fwd_args)
+
+    def backward(self, stages):
+        return self.bwd_fn(*self.bwd_args, *self.bwd_tail, stages, self.stream)
+
+
+def _check_codes(codes, fa):
+    bad = [c for c in codes if c != 0]
+    if bad:
+        raise fa.FAError(bad[0], "bench launch")
+
+
+def time_forward(prob, flush, steps, warmup, fa, keep_l2=False):
+    """Mean device time (ms) of one forward launch over `steps` launches, L2
+    flushed before each (unless keep_l2)."""
+    codes = []
+    for _ in range(warmup):
+        flush.zero_()
+        codes.append(prob.forward())
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for e0, e1 in ev:
+        if not keep_l2:
+            flush.zero_()
+        e0.record()
+        codes.append(prob.forward())
+        e1.record()
+    torch.cuda.synchronize()
+    _check_codes(codes, fa)
+    fa.check_device_status()
+    return statistics.mean(a.elapsed_time(b) for a, b in ev)
+
+
 def run_ours(args, w, world, rank, local):
     import exact_tiled_attention_35_b200 as fa
 
     dev = torch.device("cuda", torch.cuda.current_device())
-    fa.load_library()
+    lib = fa.load_library()
+    stream = torch.cuda.current_stream(dev)
+    peaks = measured_peaks()
     fwd_flops, bwd_flops = algorithmic_flops(w)
     step_flops = fwd_flops + bwd_flops
-    q, k, v, do = make_inputs(w.B, w.H, w.N, w.d, dtype=w.dtype, seed=rank, qk_gain=w.qk_gain, with_do=True)
-    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
-    o = torch.empty_like(qd)
-    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(qd), torch.empty_like(kd), torch.empty_like(vd)
-    ws = torch.empty(max(fa.workspace_size(w.B, w.H, w.N, w.d), 16), dtype=torch.uint8, device=dev)
+    prob = Problem(w, dev, rank, lib, stream)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    codes = []
 
-    def step():
-        fa.forward(qd, kd, vd, causal=w.causal, scale=w.scale, out=o, lse=lse)
+    def step(i=None, ev=None):
+        # forward, then the backward's three stages; events (when given) mark
+        # the boundaries on the launching stream
+        if ev is not None:
+            ev[0].record()
+        codes.append(prob.forward())
+        if ev is not None:
+            ev[1].record()
         if w.backward:
-            fa.backward(qd, kd, vd, o, dod, lse, causal=w.causal, scale=w.scale, dq=dq, dk=dk, dv=dv,
-                        workspace=ws)
+            for s_i, stage in enumerate((fa.STAGE_PREPROCESS, fa.STAGE_MAIN, fa.STAGE_DQ_CONVERT)):
+                codes.append(prob.backward(stage))
+                if ev is not None:
+                    ev[2 + s_i].record()
 
     for _ in range(args.warmup):
         flush.zero_()
         step()
+    torch.cuda.synchronize()
+    _check_codes(codes, fa)
     fa.check_device_status()
-    n = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+
+    # Clock soak: the same step, untimed, for about a second right before the
+    # timed steps, so the clock sampler sees the GPU under this load.
     clocks = ClockSampler(dev)
     clocks.start()
+    t_soak = time.time()
+    while time.time() - t_soak < args.soak_s:
+        for _ in range(20):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+    n = args.steps
+    nev = 5 if w.backward else 2
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(n)]
     barrier(world)
     torch.cuda.synchronize()
     for i in range(n):
         if not args.keep_l2:
             flush.zero_()  # L2 (126 MB) flushed between timed steps
-        ev[i][0].record()
-        fa.forward(qd, kd, vd, causal=w.causal, scale=w.scale, out=o, lse=lse)
-        ev[i][1].record()
-        if w.backward:
-            fa.backward(qd, kd, vd, o, dod, lse, causal=w.causal, scale=w.scale, dq=dq, dk=dk, dv=dv,
-                        workspace=ws)
-        ev[i][2].record()
+        step(i, ev[i])
     torch.cuda.synchronize()
     barrier(world)
-    clk = clocks.stop()
+    t_timed_end = time.time()
+    _check_codes(codes, fa)
     fa.check_device_status()
-    fwd_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    bwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    step_ms = statistics.mean(a + b for a, b in zip(fwd_ms, bwd_ms))
+    seg = [[e[j].elapsed_time(e[j + 1]) for e in ev] for j in range(nev - 1)]
+    fwd_ms = statistics.mean(seg[0])
+    step_ms = statistics.mean(e[0].elapsed_time(e[nev - 1]) for e in ev)
     step_ms = max_over_ranks(step_ms, world)
     value = world * step_flops / (step_ms * 1e-3) / 1e12
+    breakdown = {"forward": fwd_ms}
+    if w.backward:
+        breakdown.update({"bwd_preprocess": statistics.mean(seg[1]), "bwd_main": statistics.mean(seg[2]),
+                          "bwd_dq_convert": statistics.mean(seg[3])})
+        breakdown["backward"] = breakdown["bwd_preprocess"] + breakdown["bwd_main"] + breakdown["bwd_dq_convert"]
 
-    # end to end through the public API: pinned host inputs in, results back out
-    hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
-    ho, hlse, hdq, hdk, hdv = (torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
-                               for t in (o, lse, dq, dk, dv))
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
-    d2h = sum(t.numel() * t.element_size() for t in (ho, hlse, hdq, hdk, hdv))
-    if not w.backward:
-        h2d -= hdo.numel() * hdo.element_size()
-        d2h = ho.numel() * ho.element_size() + hlse.numel() * hlse.element_size()
+    # the dominant kernel of the step and its roofline (tensor-bound: FLOPs)
+    if w.backward and breakdown["bwd_main"] > fwd_ms:
+        dom = {"kernel": "bwd::main_kernel<%d>" % w.d, "flops": bwd_flops, "ms": breakdown["bwd_main"],
+               "timed": "the backward main kernel alone: CUDA events around its launch on the launching stream"}
+    else:
+        dom = {"kernel": "fwd::fwd_kernel<%d>" % w.d, "flops": fwd_flops, "ms": fwd_ms,
+               "timed": "the forward kernel alone: CUDA events around its launch on the launching stream"}
+    achieved = dom["flops"] / (dom["ms"] * 1e-3) / 1e12
+    roof = {"bound": "tensor", "kernel": dom["kernel"], "timed": dom["timed"], "achieved": achieved,
+            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+            "peak_source": f"{peaks['source']} bf16 burst (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
+            else "fallback bf16 burst (no MEASURED_PEAKS.json)",
+            "traffic": profiled_traffic(dom["kernel"], w.name)}
+
+    # the other workloads, forward alone, each timed the same way
+    extras = {}
+    if not args.skip_extras:
+        for key, name in (("forward_target", FWD_TARGET_WORKLOAD), ("short_seq_forward", "fwd_b4h16n1024d64"),
+                          ("long_context_forward", "fwd_b1h8n32768d128_causal_x4")):
+            ew = WORKLOADS[name]
+            ep = Problem(ew, dev, rank, lib, stream)
+            t0 = time.time()
+            ms = max_over_ranks(time_forward(ep, flush, n, args.warmup, fa), world)
+            ff = algorithmic_flops(ew, backward=False)[0]
+            tf = ff / (ms * 1e-3) / 1e12
+            rec = {"workload": name, "ms": ms, "tflops": tf, "frac_of_peak": tf / peaks["bf16_tflops"],
+                   "roofline": {"bound": "tensor", "kernel": f"fwd::fwd_kernel<{ew.d}>", "achieved": tf,
+                                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                                "frac": tf / peaks["bf16_tflops"],
+                                "traffic": profiled_traffic(f"fwd::fwd_kernel<{ew.d}>", name)}}
+            if key == "short_seq_forward":
+                hbm = (4 * ew.N * ew.d * 2 + 4 * ew.N) * ew.B * ew.H  # Q, K, V in; O, LSE out
+                rec["hbm_gbs_algorithmic"] = hbm / (ms * 1e-3) / 1e9
+                rec["hbm_frac"] = rec["hbm_gbs_algorithmic"] / peaks["hbm_gbs"]
+            extras[key] = rec
+            del ep
+        t_extras_end = time.time()
+    else:
+        t_extras_end = t_timed_end
+
+    # end to end through the public Python API: pinned host inputs in, results out
+    hq, hk, hv = (t.pin_memory() for t in prob.host[:3])
+    hdo = prob.host[3].pin_memory() if w.backward else None
+    outs = [prob.o, prob.lse] + ([prob.dq, prob.dk, prob.dv] if w.backward else [])
+    houts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv) + ((hdo,) if w.backward else ()))
+    d2h = sum(t.numel() * t.element_size() for t in houts)
 
     def e2e_step():
-        qd.copy_(hq, non_blocking=True)
-        kd.copy_(hk, non_blocking=True)
-        vd.copy_(hv, non_blocking=True)
+        prob.q.copy_(hq, non_blocking=True)
+        prob.k.copy_(hk, non_blocking=True)
+        prob.v.copy_(hv, non_blocking=True)
+        fa.forward(prob.q, prob.k, prob.v, causal=w.causal, scale=w.scale, out=prob.o, lse=prob.lse)
         if w.backward:
-            dod.copy_(hdo, non_blocking=True)
-        step()
-        ho.copy_(o, non_blocking=True)
-        hlse.copy_(lse, non_blocking=True)
-        if w.backward:
-            hdq.copy_(dq, non_blocking=True)
-            hdk.copy_(dk, non_blocking=True)
-            hdv.copy_(dv, non_blocking=True)
+            prob.do.copy_(hdo, non_blocking=True)
+            fa.backward(prob.q, prob.k, prob.v, prob.o, prob.do, prob.lse, causal=w.causal, scale=w.scale,
+                        dq=prob.dq, dk=prob.dk, dv=prob.dv, workspace=prob.ws)
+        for h, d_ in zip(houts, outs):
+            h.copy_(d_, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
         e2e_step()
@@ -340,51 +481,10 @@ def run_ours(args, w, world, rank, local):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n, world)
     barrier(world)
     fa.check_device_status()
-
-    # forward alone on the long causal workload (the tensor-peak target)
-    fw = WORKLOADS[FWD_TARGET_WORKLOAD]
-    fwd_only = None
-    if not args.skip_fwd_target:
-        fq, fk, fv = (t.to(dev) for t in make_inputs(fw.B, fw.H, fw.N, fw.d, seed=rank))
-        fo = torch.empty_like(fq)
-        flse = torch.empty((fw.B, fw.H, fw.N), dtype=torch.float32, device=dev)
-        for _ in range(args.warmup):
-            fa.forward(fq, fk, fv, causal=True, out=fo, lse=flse)
-        fev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
-        torch.cuda.synchronize()
-        for i in range(n):
-            flush.zero_()
-            fev[i][0].record()
-            fa.forward(fq, fk, fv, causal=True, out=fo, lse=flse)
-            fev[i][1].record()
-        torch.cuda.synchronize()
-        fa.check_device_status()
-        f_ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in fev), world)
-        ff = algorithmic_flops(fw, backward=False)[0]
-        fwd_only = {"workload": fw.name, "ms": f_ms, "tflops": ff / (f_ms * 1e-3) / 1e12}
-        del fq, fk, fv, fo, flse
-
-    peaks = measured_peaks()
-    fwd_avg = statistics.mean(fwd_ms)
-    bwd_avg = statistics.mean(bwd_ms) if w.backward else 0.0
-    if bwd_avg > fwd_avg:
-        dom = {"kernel": "bwd::main_kernel<%d>" % w.d, "flops": bwd_flops, "ms": bwd_avg,
-               "timed": "fa_backward as a whole: preprocess + main + dQ convert launches (the main kernel is ~83% of them in the ncu launch list), so achieved is a lower bound for the main kernel"}
-    else:
-        dom = {"kernel": "fwd::fwd_kernel<%d>" % w.d, "flops": fwd_flops, "ms": fwd_avg,
-               "timed": "fa_forward: one launch"}
-    achieved = dom["flops"] / (dom["ms"] * 1e-3) / 1e12
-    roof = {"bound": "tensor", "kernel": dom["kernel"], "timed": dom["timed"], "achieved": achieved,
-            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
-            "peak_source": peaks["source"] + " bf16 burst (MEASURED_PEAKS.json)",
-            "traffic": profiled_traffic(dom["kernel"], w.name)}
-    if fwd_only is not None:
-        fwd_only["frac_of_peak"] = fwd_only["tflops"] / peaks["bf16_tflops"]
-        fwd_only["roofline"] = {
-            "bound": "tensor", "kernel": "fwd::fwd_kernel<128>", "achieved": fwd_only["tflops"],
-            "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": fwd_only["frac_of_peak"],
-            "peak_source": peaks["source"] + " bf16 burst (MEASURED_PEAKS.json)",
-            "traffic": profiled_traffic("fwd::fwd_kernel<128>", fw.name)}
+    clocks.stop()
+    clk = clocks.summary(t_soak, t_extras_end,
+                         f"{args.soak_s:.1f} s soak of the step right before the timed steps, the timed "
+                         "steps, and the forward-only workloads after them")
 
     cpu = None
     if rank == 0 and world == 1 and not args.skip_cpu:
@@ -401,11 +501,13 @@ def run_ours(args, w, world, rank, local):
             "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
                        "global_batch": world * w.B, "seq_len": w.N, "parallelism": f"replicas{world}",
                        "l2": ("kept between timed steps (--keep-l2, a diagnostic: inputs may stay "
-                              "L2-resident)" if args.keep_l2 else "flushed between timed steps (256 MB write)")},
-            "breakdown_ms": {"forward": fwd_avg, "backward": bwd_avg},
+                              "L2-resident)" if args.keep_l2 else "flushed between timed steps (256 MB write)"),
+                       "calls": "C ABI: fa_forward, then fa_backward_stages for the preprocess, main and dQ "
+                                "convert stages (fa_backward runs the same three launches in one call)"},
+            "breakdown_ms": breakdown,
             "frac_of_peak": value / world / peaks["bf16_tflops"],
             "roofline": roof,
-            "forward_target": fwd_only,
+            **extras,
             "cpu_baseline": cpu,
             "e2e": {"value": world * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
@@ -424,7 +526,10 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle CPU work")
     ap.add_argument("--skip-cpu", action="store_true")
-    ap.add_argument("--skip-fwd-target", action="store_true")
+    ap.add_argument("--skip-extras", action="store_true",
+                    help="skip the forward-only timings of the other workloads")
+    ap.add_argument("--soak-s", type=float, default=1.0,
+                    help="seconds of untimed steps right before the timed ones (clock sampling)")
     ap.add_argument("--keep-l2", action="store_true",
                     help="do not flush L2 between timed steps (diagnostic for the small workloads; "
                          "the default flushes)")

@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   // whole opt-in shared memory, so there is no slack to re-align: refuse to run
   // on a misaligned base instead of computing garbage.
   if (smem_u32(smem) & 1023u) {
-    if (threadIdx.x == 0) atomicCAS(&g_device_status, 0u, 0x200u);
+    if (threadIdx.x == 0) record_state_error(kStateMisalignedSmem);
     return;
   }
   uint8_t* sK = smem + C::OFF_K;
@@ -564,7 +564,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 }
 
 // -D, -LSE*log2(e) (padded; the main kernel adds them) and a zeroed dQ
-// accumulator; one warp per padded row.
+// accumulator.  A row of O and dO is D/8 lanes' worth of 16-byte loads, so a
+// warp covers 256/D rows at once; every access is a 16-byte vector.
 template <int D>
 __global__ void __launch_bounds__(256) preprocess_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dout,
@@ -573,48 +574,61 @@ __global__ void __launch_bounds__(256) preprocess_kernel(const __nv_bfloat16* __
                                                          float* __restrict__ dsum,
                                                          float* __restrict__ dq_acc, int BH, int N,
                                                          int Npad) {
-  const long long gw = (long long)blockIdx.x * 8 + threadIdx.x / 32;
+  constexpr int L = D / 8;          // lanes per row
+  constexpr int RPW = 32 / L;       // rows per warp
   const int lane = threadIdx.x % 32;
-  if (gw >= (long long)BH * Npad) return;
-  const int bh = (int)(gw / Npad), row = (int)(gw % Npad);
-  if (row >= N) {
-    if (lane == 0) {
-      lse2[gw] = -INFINITY;  // padding rows: probability exp2(-inf) = 0
-      dsum[gw] = 0.f;
-    }
-    return;
-  }
-  const size_t off = ((size_t)bh * N + row) * D;
+  const long long gr = ((long long)blockIdx.x * 8 + threadIdx.x / 32) * RPW + lane / L;
+  if (gr >= (long long)BH * Npad) return;
+  const int bh = (int)(gr / Npad), row = (int)(gr % Npad);
+  const int c = (lane % L) * 8;
   float acc = 0.f;
+  if (row < N) {
+    const size_t off = ((size_t)bh * N + row) * D + c;
+    const uint4 a = *reinterpret_cast<const uint4*>(o + off);
+    const uint4 g = *reinterpret_cast<const uint4*>(dout + off);
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
 #pragma unroll
-  for (int c = lane * 2; c < D; c += 64) {
-    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(o + off + c);
-    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(dout + off + c);
-    acc = fmaf(__low2float(a), __low2float(b), acc);
-    acc = fmaf(__high2float(a), __high2float(b), acc);
+    for (int i = 0; i < 4; ++i) {
+      const float2 af = __bfloat1622float2(a2[i]), gf = __bfloat1622float2(g2[i]);
+      acc = fmaf(af.x, gf.x, acc);
+      acc = fmaf(af.y, gf.y, acc);
+    }
+    float4* z = reinterpret_cast<float4*>(dq_acc + off);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  // the L lanes of a row are consecutive and L-aligned: reduce within them
 #pragma unroll
-  for (int sh = 16; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
-  float4* z = reinterpret_cast<float4*>(dq_acc + off);
-  for (int c = lane; c < D / 4; c += 32) z[c] = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (lane == 0) {
-    dsum[gw] = -acc;
-    // a row that saw no key in the forward (LSE = -inf) gets probability 0 too
-    const float l = lse[(size_t)bh * N + row];
-    lse2[gw] = l == -INFINITY ? -INFINITY : -l * kLog2e;
+  for (int sh = L / 2; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+  if (lane % L == 0) {
+    if (row >= N) {
+      lse2[gr] = -INFINITY;  // padding rows: probability exp2(-inf) = 0
+      dsum[gr] = 0.f;
+    } else {
+      dsum[gr] = -acc;
+      // a row that saw no key in the forward (LSE = -inf) gets probability 0 too
+      const float l = lse[(size_t)bh * N + row];
+      lse2[gr] = l == -INFINITY ? -INFINITY : -l * kLog2e;
+    }
   }
 }
 
+// dQ = scale * accumulator in bf16: eight values per thread (two 16-byte loads,
+// one 16-byte store).
 __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict__ acc,
-                                                         __nv_bfloat16* __restrict__ dq, long long n4,
+                                                         __nv_bfloat16* __restrict__ dq, long long n8,
                                                          float scale) {
-  for (long long idx = (long long)blockIdx.x * 256 + threadIdx.x; idx < n4;
+  for (long long idx = (long long)blockIdx.x * 256 + threadIdx.x; idx < n8;
        idx += (long long)gridDim.x * 256) {
-    const float4 a = reinterpret_cast<const float4*>(acc)[idx];
-    uint2 w;
+    const float4 a = reinterpret_cast<const float4*>(acc)[2 * idx];
+    const float4 b = reinterpret_cast<const float4*>(acc)[2 * idx + 1];
+    uint4 w;
     w.x = pack_bf16x2(a.x * scale, a.y * scale);
     w.y = pack_bf16x2(a.z * scale, a.w * scale);
-    reinterpret_cast<uint2*>(dq)[idx] = w;
+    w.z = pack_bf16x2(b.x * scale, b.y * scale);
+    w.w = pack_bf16x2(b.z * scale, b.w * scale);
+    reinterpret_cast<uint4*>(dq)[idx] = w;
   }
 }
 
@@ -651,7 +665,8 @@ cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const C
                            const CUtensorMap& mdo, const CUtensorMap& mdq, const void* o,
                            const void* dout, const float* lse,
                            void* dq, void* dk, void* dv, void* workspace, int B, int H, int Hkv,
-                           int Nq, int Nk, int d, float scale, int causal, cudaStream_t st) {
+                           int Nq, int Nk, int d, float scale, int causal, int stages,
+                           cudaStream_t st) {
   const int BH = B * H;
   const int N = Nq;  // the workspace and the preprocess run over query rows
   const int npad = (N + 127) / 128 * 128;
@@ -659,16 +674,21 @@ cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const C
   float* lse2 = static_cast<float*>(workspace);
   float* dsum = reinterpret_cast<float*>(static_cast<char*>(workspace) + vec);
   float* acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * vec);
-  const long long rows = (long long)BH * npad;
-  const unsigned pblocks = (unsigned)((rows + 7) / 8);
-  if (d == 128)
-    bwd::preprocess_kernel<128><<<pblocks, 256, 0, st>>>(
-        (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, lse2, dsum, acc, BH, N, npad);
-  else
-    bwd::preprocess_kernel<64><<<pblocks, 256, 0, st>>>(
-        (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, lse2, dsum, acc, BH, N, npad);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (stages & kStagePreprocess) {
+    const long long rows = (long long)BH * npad;
+    const long long rows_per_block = 8LL * (256 / d);  // 8 warps of 256/d rows
+    const unsigned pblocks = (unsigned)((rows + rows_per_block - 1) / rows_per_block);
+    if (d == 128)
+      bwd::preprocess_kernel<128><<<pblocks, 256, 0, st>>>(
+          (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, lse2, dsum, acc, BH, N, npad);
+    else
+      bwd::preprocess_kernel<64><<<pblocks, 256, 0, st>>>(
+          (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, lse2, dsum, acc, BH, N, npad);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (!(stages & (kStageMain | kStageConvert))) return cudaSuccess;
 
   bwd::Params p;
   p.dk = static_cast<__nv_bfloat16*>(dk);
@@ -694,7 +714,8 @@ cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const C
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   p.chunk = bwd::chunk_heads(p.BHkv, p.G, Nq, Nk, d, p.nkv, std::max(sms, 1));
   const dim3 grid((unsigned)(p.nkv * p.BHkv));
-  if (d == 128) {
+  if (!(stages & kStageMain)) {
+  } else if (d == 128) {
     const int smem = bwd::Cfg<128>::SMEM_BYTES;
     e = cudaFuncSetAttribute(bwd::main_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -706,10 +727,10 @@ cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const C
     bwd::main_kernel<64><<<grid, bwd::NTHREADS, smem, st>>>(mq, mk, mv, mdo, mdq, p);
   }
   e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const long long n4 = (long long)BH * N * d / 4;
-  const unsigned cblocks = (unsigned)std::min<long long>((n4 + 255) / 256, 148LL * 16);
-  bwd::dq_convert_kernel<<<cblocks, 256, 0, st>>>(acc, static_cast<__nv_bfloat16*>(dq), n4, scale);
+  if (e != cudaSuccess || !(stages & kStageConvert)) return e;
+  const long long n8 = (long long)BH * N * d / 8;
+  const unsigned cblocks = (unsigned)std::min<long long>((n8 + 255) / 256, (long long)std::max(sms, 1) * 8);
+  bwd::dq_convert_kernel<<<cblocks, 256, 0, st>>>(acc, static_cast<__nv_bfloat16*>(dq), n8, scale);
   return cudaGetLastError();
 }
 

@@ -27,8 +27,20 @@ __device__ __forceinline__ unsigned long long global_timer_ns() {
   return t;
 }
 
+// Status word codes: 0x100 | site = a bounded wait at `site` ran out;
+// kStateError | cause = a kernel found device-side state it cannot trust and
+// skipped work.  Only the first error since the last read is kept.
+constexpr unsigned int kTimeoutError = 0x100u;
+constexpr unsigned int kStateError = 0x200u;
+constexpr unsigned int kStateMisalignedSmem = 0x01u;  // dynamic shared memory base
+constexpr unsigned int kStateTicketOwner = 0x02u;     // scheduler slot held by another launch
+
 __device__ __forceinline__ void record_timeout(unsigned int site) {
-  atomicCAS(&g_device_status, 0u, 0x100u | site);
+  atomicCAS(&g_device_status, 0u, kTimeoutError | (site & 0xFFu));
+}
+
+__device__ __forceinline__ void record_state_error(unsigned int cause) {
+  atomicCAS(&g_device_status, 0u, kStateError | cause);
 }
 
 // ----------------------------------------------------------------- mbarrier
@@ -150,6 +162,27 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       : "memory");
 }
 
+// The same two forms with kind::f8f6f4 (here: e4m3 A and B, fp32 accumulate).
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05.mma issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile(
@@ -171,25 +204,6 @@ __device__ __forceinline__ void tmem_wait_st() {
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
-      "[%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-        "=r"(r[31])
-      : "r"(taddr));
-}
-
-// Warp loads 16 lanes x 64 columns (shape 16x256b, 8 repetitions along the
-// columns).  Thread t receives, for column block j (8 columns each), r[4j], r[4j+1]
-// = lane base + t/4, columns 8j + 2(t%4) and 8j + 2(t%4) + 1, and r[4j+2], r[4j+3]
-// = the same columns of lane base + 8 + t/4.
-__device__ __forceinline__ void tmem_ld16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
       "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
       "[%32];"
@@ -229,12 +243,18 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 
 // ------------------------------------------------------- UMMA descriptors
 
-// Shared-memory matrix descriptor, 128-byte swizzle (the layout TMA writes with
-// CU_TENSOR_MAP_SWIZZLE_128B): start address, leading and stride byte offsets
-// (all >> 4), descriptor version 1, layout type 2 = SWIZZLE_128B.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// Shared-memory matrix descriptor for a swizzled layout (the one TMA writes with
+// CU_TENSOR_MAP_SWIZZLE_128B or _64B): start address, leading and stride byte
+// offsets (all >> 4), descriptor version 1, and the layout type, 2 = 128-byte
+// swizzle, 4 = 64-byte swizzle.
+__device__ __forceinline__ uint64_t sdesc_swz(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                              uint32_t layout) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
+}
+
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return sdesc_swz(saddr, lbo, sbo, 2u);
 }
 
 // The same descriptor for an operand `bytes` further on in shared memory.  The
@@ -259,6 +279,17 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
   return (1u << 4)                      // D format: f32
          | (1u << 7)                    // A format: bf16
          | (1u << 10)                   // B format: bf16
+         | ((uint32_t)a_mn << 15)       // A major
+         | ((uint32_t)b_mn << 16)       // B major
+         | ((uint32_t)(N >> 3) << 17)   // N / 8
+         | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+// Instruction descriptor, kind::f8f6f4 with e4m3 A/B (format code 0) and fp32 D.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4)                      // D format: f32
+         | (0u << 7)                    // A format: e4m3
+         | (0u << 10)                   // B format: e4m3
          | ((uint32_t)a_mn << 15)       // A major
          | ((uint32_t)b_mn << 16)       // B major
          | ((uint32_t)(N >> 3) << 17)   // N / 8
@@ -301,6 +332,41 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// Two fp32 values to e4m3 (round to nearest even, saturating to +-448): lo in
+// bits 0-7, hi in bits 8-15.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return (uint32_t)r;
+}
+
+// exp2 of two values on the FMA pipe instead of the MUFU unit, for part of the
+// exponentials (the two units then share the work).  Cody-Waite range
+// reduction: n = round(x) and f = x - n in [-1/2, 1/2] (one add of 1.5 * 2^23
+// leaves n in the low mantissa bits; subtracting it again gives n exactly), then
+// 2^f by a degree-3 polynomial whose coefficients are the float32 rounding of
+// the minimax (Remez) fit of relative error on [-1/2, 1/2] (csrc/exp2_poly_fit.py;
+// maximum relative error 7.5e-5), and finally n is added to the exponent field.
+// x is clamped at -120 first, so -inf and large negative inputs give about
+// 2^-120 rather than 0: callers use it only where no element is masked.
+__device__ __forceinline__ void ex2_poly_x2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0x1.fff692p-1f, c1 = 0x1.62f31ap-1f, c2 = 0x1.f0de1ap-3f, c3 = 0x1.c3f76p-5f;
+  const uint64_t x = f2_pack(fmaxf(x0, -120.f), fmaxf(x1, -120.f));
+  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));
+  const uint64_t n = f2_add(t, f2_pack(-kRound, -kRound));
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);
+  uint64_t q = f2_fma(f2_pack(c3, c3), f, f2_pack(c2, c2));
+  q = f2_fma(q, f, f2_pack(c1, c1));
+  q = f2_fma(q, f, f2_pack(c0, c0));
+  float t0, t1, q0, q1;
+  f2_unpack(t, t0, t1);
+  f2_unpack(q, q0, q1);
+  // q * 2^n: the low bits of t hold n; shifted to the exponent field they add n
+  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

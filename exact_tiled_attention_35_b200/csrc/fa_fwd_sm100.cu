@@ -39,6 +39,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <type_traits>
 
 #include "fa_device.cuh"
 #include "fa_kernels.h"
@@ -55,6 +56,7 @@ constexpr int kMmaWarp = 9;
 constexpr int kItemRing = 2;       // work items the producer may hand out ahead
 constexpr int kItemReaders = 9;    // MMA issuer and the 8 softmax warps
 constexpr int kSchedSlots = 256;   // ticket counters, one per launch in flight
+constexpr unsigned int kHeldTag = 0xFFFFFFFFu;  // owner tag of no launch (diagnostics)
 // Register split (setmaxnreg).  The launch gives every thread 168 registers,
 // 384 * 168 = 64512 in all; the shares sum to 128 * (2*208 + 88) = 64512.
 constexpr int kRegsSoftmax = 208;  // warpgroups 0 and 1
@@ -64,18 +66,37 @@ static_assert(128 * (2 * kRegsSoftmax + kRegsControl) <= NTHREADS * 168,
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
-template <int D>
+// Exponentials of unmasked tiles computed on the FMA pipe (ex2_poly_x2) rather
+// than the MUFU unit: this many of every 8 pairs of a row's keys.
+constexpr int kEmuPairsPer8 = 0;
+
+// Tile geometry for head dimension D and element type (F8: e4m3, else bf16).
+// A 128-row tile is stored as NCHUNK column chunks of SW bytes per row, each in
+// the SW-byte swizzled layout TMA writes (SW = 128, or 64 for e4m3 with D = 64).
+template <int D, bool F8>
 struct Cfg {
-  static constexpr int TILE = BN * D * 2;          // bytes of one 128-row bf16 tile
-  static constexpr int CHUNK = BN * 128;           // bytes of one 64-column swizzle chunk
-  static constexpr int NSLOT = D == 128 ? 5 : 10;  // K/V ring slots
+  static constexpr int EB = F8 ? 1 : 2;                 // bytes per element
+  static constexpr int ROWB = D * EB;                   // bytes per tile row
+  static constexpr int SW = ROWB < 128 ? ROWB : 128;    // swizzle span
+  static constexpr int NCHUNK = ROWB / SW;
+  static constexpr int CHUNK = BN * SW;                 // bytes of one column chunk
+  static constexpr int TILE = BN * ROWB;                // bytes of one 128-row tile
+  static constexpr uint32_t LAYOUT = SW == 128 ? 2u : 4u;  // descriptor layout type
+  static constexpr int SBO = 8 * SW;                    // 8-row group stride
+  static constexpr int KSTEP = 32 / EB;                 // K elements per MMA (32 bytes)
+  static constexpr int S_STEPS = D / KSTEP;             // MMAs per S tile
+  static constexpr int PV_STEPS = BN / KSTEP;           // MMAs per P V (all 128 keys)
+  static constexpr int PCOLS = BN * EB / 4;             // tensor-memory columns of P
+  static constexpr int NSLOT = F8 ? (D == 128 ? 12 : 16) : (D == 128 ? 5 : 10);  // K/V ring slots
   static constexpr int SMEM_Q = NQT * TILE;
   static constexpr int SMEM_RING = NSLOT * TILE;
   static constexpr int OFF_BAR = SMEM_Q + SMEM_RING;
   static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;  // barriers + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, 0, 0);
-  static constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, 0, 1);
+  static constexpr uint32_t IDESC_QK = F8 ? idesc_e4m3(BM, BN, 0, 0) : idesc_bf16(BM, BN, 0, 0);
+  static constexpr uint32_t IDESC_PV = F8 ? idesc_e4m3(BM, D, 0, 1) : idesc_bf16(BM, D, 0, 1);
+  static_assert(SMEM_BYTES <= 232448, "shared memory over the per-block limit");
+  static_assert(NSLOT <= 16, "K/V ring larger than its barrier arrays");
 };
 
 struct Params {
@@ -91,8 +112,10 @@ struct Params {
   int chunk;   // query heads per locality chunk (their K/V stay resident in L2)
   int items;   // work items = query-tile pairs x heads
   int slot;    // ticket counter of this launch
-  float scale;
-  float scale_log2;
+  unsigned int tag;  // this launch's owner tag for the slot (nonzero)
+  float scale;       // multiplies the stored Q K^T to give the scores (LSE)
+  float scale_log2;  // the same times log2(e)
+  float o_scale;     // multiplies P V / l (the stored V's scale; 1 for bf16)
   int causal;
 };
 
@@ -112,13 +135,26 @@ struct Bars {
   uint32_t tmem_base;
 };
 
-// Ticket counters of the work-item scheduler: [slot][0] hands out work items past
-// the first gridDim.x, [slot][1] counts CTAs that have drawn their last ticket.
-// The last such CTA of a launch sets both back to zero, so the next launch that
-// draws the same slot starts clean.  The host draws slots round-robin; two launches in flight
-// at the same time on one device share a slot only if kSchedSlots launches were
-// issued in between.
-__device__ unsigned int g_fwd_tickets[kSchedSlots][2];
+// Ticket counters of the work-item scheduler, three words per slot: [0] hands
+// out work items past the first gridDim.x, [1] counts CTAs that have drawn
+// their last ticket, [2] holds the owner tag of the launch using the slot (0 =
+// free).  Every launch carries a nonzero tag of its own, and each CTA claims the
+// slot for it (compare-and-swap from 0, or finding its own tag) once, before its
+// first draw; a slot left held by a launch that never finished, or shared with a
+// launch still in flight, fails the claim and is reported (kStateTicketOwner in
+// the status word) instead of handing out wrong items.  The draws themselves are
+// single atomic adds.  The last CTA of a launch zeroes the counters, then frees
+// the tag.  The host draws slots round-robin.
+__device__ unsigned long long g_fwd_tickets[kSchedSlots][3];
+
+// Claims the slot for the launch tagged `tag`; false (recorded) if another
+// launch holds it.
+__device__ __forceinline__ bool ticket_claim(unsigned long long* slot, unsigned int tag) {
+  const unsigned long long old = atomicCAS(slot + 2, 0ull, (unsigned long long)tag);
+  if (old == 0ull || old == (unsigned long long)tag) return true;
+  record_state_error(kStateTicketOwner);
+  return false;
+}
 
 // Number of key tiles the query tile starting at row q0 needs: 0 past the last
 // query, and 0 too when the causal mask hides every key from every row of the
@@ -145,11 +181,11 @@ __device__ __forceinline__ void decode_item(const Params& p, int item, int& bh, 
   pair = p.causal ? (p.npairs - 1 - rank) : rank;
 }
 
-template <int D>
+template <int D, bool F8>
 __global__ void __launch_bounds__(NTHREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                const __grid_constant__ CUtensorMap mv, const Params p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sQ = smem;
@@ -223,14 +259,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
    if (warp == kProducerWarp) {
     if (lane == 0) {
       bool ok = true;
+      bool owner = true;      // false if the slot turned out to be held by another launch
+      bool claimed = false;
       int gseq = 0;           // K/V ring position, continued across items
       int qcnt[NQT] = {0, 0};  // Q_t loads so far
-      unsigned int* tickets = &g_fwd_tickets[p.slot][0];
+      unsigned long long* tickets = &g_fwd_tickets[p.slot][0];
       for (int r = 0; ok; ++r) {
         // The first item of CTA b is b; each later one is drawn from the launch's
         // ticket counter once this CTA's loads for the previous one are issued, so
-        // a CTA takes new work about when it is about to run out of it.
-        const int item = r == 0 ? (int)blockIdx.x : (int)gridDim.x + (int)atomicAdd(tickets, 1u);
+        // a CTA takes new work about when it is about to run out of it.  A slot
+        // held by another launch ends this CTA's work (and is reported).
+        int item = (int)blockIdx.x;
+        if (r == 1) {
+          owner = ticket_claim(tickets, p.tag);
+          claimed = true;
+        }
+        if (r > 0) item = owner ? (int)gridDim.x + (int)atomicAdd(tickets, 1ull) : p.items;
         const int s = r % kItemRing;
         if (r >= kItemRing) ok = mbar_wait(&bars->it_empty[s], (uint32_t)((r / kItemRing - 1) & 1), 24);
         if (!ok) break;
@@ -243,8 +287,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (qcnt[t] > 0) ok = mbar_wait(&bars->q_empty[t], (qcnt[t] - 1) & 1, 10);
           if (!ok) break;
           mbar_arrive_expect_tx(&bars->q_full[t], C::TILE);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &mq, &bars->q_full[t], c * 64,
+          for (int c = 0; c < C::NCHUNK; ++c)
+            tma_load_3d(sQ + t * C::TILE + c * C::CHUNK, &mq, &bars->q_full[t], c * (C::SW / C::EB),
                         w.qbase + t * BM, w.bh);
           ++qcnt[t];
         }
@@ -258,17 +302,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           const CUtensorMap* m = (s2 & 1) ? &mv : &mk;
           uint8_t* dst = sRing + slot * C::TILE;
           mbar_arrive_expect_tx(&bars->kv_full[slot], C::TILE);
-          for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(dst + c * C::CHUNK, m, &bars->kv_full[slot], c * 64, j * BN, w.bkv);
+          for (int c = 0; c < C::NCHUNK; ++c)
+            tma_load_3d(dst + c * C::CHUNK, m, &bars->kv_full[slot], c * (C::SW / C::EB), j * BN, w.bkv);
         }
         gseq += 2 * w.nmax;
       }
       // This CTA draws no more tickets (it has drawn one past the last item, or
-      // given up on a wait); the last CTA to get here resets the slot.
+      // given up on a wait); the last CTA to get here frees the slot.  A CTA that
+      // gave up before its first draw still claims the slot, so the count of
+      // CTAs done stays that of the launch.
+      if (!claimed) owner = ticket_claim(tickets, p.tag);
       __threadfence();
-      if (atomicAdd(tickets + 1, 1u) == gridDim.x - 1) {
-        atomicExch(tickets, 0u);
-        atomicExch(tickets + 1, 0u);
+      if (owner && atomicAdd(tickets + 1, 1ull) == (unsigned long long)gridDim.x - 1) {
+        atomicExch(tickets, 0ull);
+        atomicExch(tickets + 1, 0ull);
+        __threadfence();
+        atomicExch(tickets + 2, 0ull);
       }
       // make sure no copy into this CTA's shared memory is still in flight at exit
       for (int slot = 0; slot < C::NSLOT && slot < gseq; ++slot) {
@@ -286,30 +335,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       // spends few instructions per MMA.
       // One descriptor for the start of shared memory (Q_0, K-major); the ring
       // follows the Q tiles, and an MN-major operand differs only in LBO.
-      const uint64_t d0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t d0 = sdesc_swz(smem_u32(sQ), 16, C::SBO, C::LAYOUT);
       constexpr uint64_t kToMn = (uint64_t)((C::CHUNK >> 4) - 1) << 16;  // LBO 16 B -> CHUNK
-      // S_t = Q_t K_j^T : A = Q_t (K-major), B = K_j (K-major), K = D in steps of 16
+      // S_t = Q_t K_j^T : A = Q_t (K-major), B = K_j (K-major), K = D in steps of 32 bytes
       auto issue_s = [&](int t, uint32_t kslot) {
         const uint64_t d = opaque(d0);
         const uint64_t a = sdesc_at(d, t * C::TILE), b = sdesc_at(d, C::SMEM_Q + kslot * C::TILE);
         const uint32_t d_tmem = tmem + t * BN;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t koff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_ss(d_tmem, sdesc_at(a, koff), sdesc_at(b, koff), C::IDESC_QK, kk > 0);
+        for (int kk = 0; kk < C::S_STEPS; ++kk) {
+          const uint32_t koff = ((kk * 32) / C::SW) * C::CHUNK + (kk * 32) % C::SW;
+          if constexpr (F8)
+            mma_ss_f8(d_tmem, sdesc_at(a, koff), sdesc_at(b, koff), C::IDESC_QK, kk > 0);
+          else
+            mma_ss(d_tmem, sdesc_at(a, koff), sdesc_at(b, koff), C::IDESC_QK, kk > 0);
         }
       };
-      // O_t += P_t V_j : A = P_t (tensor memory), B = V_j (MN-major), K = 128 keys,
-      // issued in two halves (keys 0-63, 64-127) as the softmax group publishes them
+      // O_t += P_t V_j : A = P_t (tensor memory, 8 columns per 32 bytes of keys),
+      // B = V_j (MN-major), K = 128 keys, issued in two halves (keys 0-63, 64-127)
+      // as the softmax group publishes them
       auto issue_pv = [&](int t, uint32_t vslot, int j, int half) {
         const uint64_t b = sdesc_at(opaque(d0), C::SMEM_Q + vslot * C::TILE) + kToMn;
         const uint32_t d_tmem = tmem + 2 * BN + t * D;
         const uint32_t a_tmem = tmem + t * BN;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int kk = half * 4 + q;
-          mma_ts(d_tmem, a_tmem + kk * 8, sdesc_at(b, kk * 16 * 128), C::IDESC_PV,
-                 (j > 0 || kk > 0) ? 1u : 0u);
+        for (int q = 0; q < C::PV_STEPS / 2; ++q) {
+          const int kk = half * (C::PV_STEPS / 2) + q;
+          if constexpr (F8)
+            mma_ts_f8(d_tmem, a_tmem + kk * 8, sdesc_at(b, kk * C::KSTEP * C::SW), C::IDESC_PV,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+          else
+            mma_ts(d_tmem, a_tmem + kk * 8, sdesc_at(b, kk * C::KSTEP * C::SW), C::IDESC_PV,
+                   (j > 0 || kk > 0) ? 1u : 0u);
         }
       };
       auto advance = [](uint32_t& slot, uint32_t& phase) {
@@ -474,21 +531,48 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const float mc = m_used == -INFINITY ? 0.f : m_used * c;
       const uint64_t c2 = f2_pack(c, c), nmc2 = f2_pack(-mc, -mc);
       uint64_t sum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+      // Exponentials of one half (64 keys), packed for the P V MMA (bf16 pairs, or
+      // e4m3 quadruples); in a tile without masked keys some pairs are computed on
+      // the FMA pipe, spread evenly over the row.
+      auto exps = [&](auto emu, int half, uint32_t(&pk)[32]) {
+        constexpr bool kEmu = decltype(emu)::value;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int e = half * 64 + 2 * i;
+          float x0, x1, p0, p1;
+          f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), c2, nmc2), x0, x1);
+          if (kEmu && ((i * kEmuPairsPer8) % 8) < kEmuPairsPer8) {
+            ex2_poly_x2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2(x0);
+            p1 = ex2(x1);
+          }
+          sum2[i % 2] = f2_add(sum2[i % 2], f2_pack(p0, p1));
+          if constexpr (F8) {
+            const uint32_t h = pack_e4m3x2(p0, p1);
+            pk[i / 2] = (i % 2) ? (pk[i / 2] | (h << 16)) : h;
+          } else {
+            pk[i] = pack_bf16x2(p0, p1);
+          }
+        }
+      };
       // Exponentials in two halves of 64 keys; each half goes to tensor memory and
       // is published at once so the P V MMA can start on it.
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
+        if (need_mask)
+          exps(std::false_type{}, half, pk);
+        else
+          exps(std::true_type{}, half, pk);
+        if constexpr (F8) {
+          uint32_t pk16[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int e = half * 64 + 2 * i;
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), c2, nmc2), x0, x1);
-          const float p0 = ex2(x0), p1 = ex2(x1);
-          sum2[i % 2] = f2_add(sum2[i % 2], f2_pack(p0, p1));
-          pk[i] = pack_bf16x2(p0, p1);
+          for (int i = 0; i < 16; ++i) pk16[i] = pk[i];
+          tmem_st16(tS + half * 16, pk16);
+        } else {
+          tmem_st32(tS + half * 32, pk);
         }
-        tmem_st32(tS + half * 32, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(half ? &bars->p_hi[t] : &bars->p_lo[t]);
@@ -501,7 +585,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (ok) ok = mbar_wait(&bars->o_full[t], icnt & 1, 20 + t);
     if (ok) {
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = l > 0.f ? p.o_scale / l : 0.f;
       __nv_bfloat16* orow = p.o + ((size_t)bh * p.Nq + (size_t)(q_row < p.Nq ? q_row : 0)) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -534,13 +618,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-// Query heads per locality chunk.  A chunk's K and V (4 N d bytes per key/value
+// Query heads per locality chunk.  A chunk's K and V (2 N row_bytes per key/value
 // head) should fit in about 40 MB of the 126 MB L2, a chunk should hold at least
 // two items per CTA so that its light tail balances the CTAs, chunks split the
 // heads evenly, and a group of query heads sharing a key/value head never
 // straddles two chunks.
-inline int chunk_heads(int BH, int G, int N, int d, int npairs, int grid) {
-  const long long kv_head = 4LL * N * d;
+inline int chunk_heads(int BH, int G, int N, int row_bytes, int npairs, int grid) {
+  const long long kv_head = 2LL * N * row_bytes;
   long long c = std::max(1LL, (40LL << 20) / kv_head) * G;
   c = std::max<long long>(c, (2LL * grid + npairs - 1) / npairs);
   c = std::min<long long>(((c + G - 1) / G) * G, BH);
@@ -552,9 +636,48 @@ inline int chunk_heads(int BH, int G, int N, int d, int npairs, int grid) {
 
 }  // namespace fwd
 
+namespace fwd {
+// Marks every scheduler slot as held by a launch that never finishes (owner tag
+// kHeldTag, which no launch is given).
+__global__ void hold_scheduler_kernel() {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < kSchedSlots) {
+    g_fwd_tickets[i][0] = 0ull;
+    g_fwd_tickets[i][1] = 0ull;
+    g_fwd_tickets[i][2] = (unsigned long long)kHeldTag;
+  }
+}
+}  // namespace fwd
+
+cudaError_t sm100_forward_hold_scheduler(cudaStream_t st) {
+  fwd::hold_scheduler_kernel<<<1, fwd::kSchedSlots, 0, st>>>();
+  return cudaGetLastError();
+}
+
+cudaError_t sm100_forward_reset_scheduler() {
+  static const unsigned long long zeros[fwd::kSchedSlots][3] = {};
+  return cudaMemcpyToSymbol(fwd::g_fwd_tickets, zeros, sizeof(zeros));
+}
+
+namespace {
+
+template <int D, bool F8>
+cudaError_t launch_fwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const fwd::Params& p, cudaStream_t st) {
+  const int smem = fwd::Cfg<D, F8>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(fwd::fwd_kernel<D, F8>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  fwd::fwd_kernel<D, F8><<<grid, fwd::NTHREADS, smem, st>>>(mq, mk, mv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                           void* o, float* lse, int B, int H, int Hkv, int Nq, int Nk, int d,
-                          float scale, int causal, cudaStream_t st) {
+                          float scale, int causal, bool fp8, float qk_descale, float v_descale,
+                          cudaStream_t st) {
   const int BH = B * H;
   fwd::Params p;
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -566,8 +689,9 @@ cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   p.Nk = Nk;
   p.off = Nk - Nq;
   p.npairs = (Nq + 2 * fwd::BM - 1) / (2 * fwd::BM);
-  p.scale = scale;
-  p.scale_log2 = scale * fwd::kLog2e;
+  p.scale = scale * qk_descale;
+  p.scale_log2 = p.scale * fwd::kLog2e;
+  p.o_scale = v_descale;
   p.causal = causal;
   p.items = p.npairs * BH;
   // persistent: one CTA per SM, each taking items as it becomes free
@@ -575,22 +699,16 @@ cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   if (cudaGetDevice(&dev) == cudaSuccess)
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const dim3 grid((unsigned)std::min(p.items, std::max(sms, 1)));
-  p.chunk = fwd::chunk_heads(BH, p.G, Nk, d, p.npairs, (int)grid.x);
-  static std::atomic<unsigned int> launches{0};
-  p.slot = (int)(launches.fetch_add(1u, std::memory_order_relaxed) % fwd::kSchedSlots);
-  cudaError_t e;
-  if (d == 128) {
-    const int smem = fwd::Cfg<128>::SMEM_BYTES;
-    e = cudaFuncSetAttribute(fwd::fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    fwd::fwd_kernel<128><<<grid, fwd::NTHREADS, smem, st>>>(mq, mk, mv, p);
-  } else {
-    const int smem = fwd::Cfg<64>::SMEM_BYTES;
-    e = cudaFuncSetAttribute(fwd::fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    fwd::fwd_kernel<64><<<grid, fwd::NTHREADS, smem, st>>>(mq, mk, mv, p);
-  }
-  return cudaGetLastError();
+  p.chunk = fwd::chunk_heads(BH, p.G, Nk, d * (fp8 ? 1 : 2), p.npairs, (int)grid.x);
+  static std::atomic<unsigned long long> launches{0};
+  const unsigned long long seq = launches.fetch_add(1ull, std::memory_order_relaxed);
+  p.slot = (int)(seq % fwd::kSchedSlots);
+  p.tag = (unsigned int)(seq % (unsigned long long)(fwd::kHeldTag - 1u)) + 1u;  // 1 .. kHeldTag-1
+  if (fp8)
+    return d == 128 ? launch_fwd<128, true>(grid, mq, mk, mv, p, st)
+                    : launch_fwd<64, true>(grid, mq, mk, mv, p, st);
+  return d == 128 ? launch_fwd<128, false>(grid, mq, mk, mv, p, st)
+                  : launch_fwd<64, false>(grid, mq, mk, mv, p, st);
 }
 
 }  // namespace fa

@@ -20,9 +20,22 @@ cudaError_t simt_backward(bool bf16, const void* q, const void* k, const void* v
 // with a {64, 128, 1} box and 128-byte swizzle.  Hkv divides H (Hkv = H: plain
 // multi-head attention).  Under the causal mask key j is visible to query i iff
 // j <= i + Nk - Nq.
+// fp8: Q, K, V are e4m3 (maps of uint8 elements, box {min(d, 128), 128, 1}, swizzle
+// of min(d, 128) bytes); the scores are scale * qk_descale * (Q K^T of the stored
+// values) and O = v_descale * P V / l.  bf16: qk_descale = v_descale = 1.
 cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                           void* o, float* lse, int B, int H, int Hkv, int Nq, int Nk, int d,
-                          float scale, int causal, cudaStream_t st);
+                          float scale, int causal, bool fp8, float qk_descale, float v_descale,
+                          cudaStream_t st);
+
+// Frees every slot of the forward's work-item scheduler on the current device
+// (synchronous).  Only for recovery after a reported device error, with no
+// forward launch in flight.
+cudaError_t sm100_forward_reset_scheduler();
+// Diagnostic: enqueues on `st` a write that marks every scheduler slot as held by
+// a launch that never finishes, so the next forward launch reports
+// kStateTicketOwner instead of computing.
+cudaError_t sm100_forward_hold_scheduler(cudaStream_t st);
 
 // tcgen05 backward (fa_bwd_sm100.cu): preprocess, main and dQ-convert kernels.
 // Workspace layout (N = query rows): LSE*log2(e) [BH, Npad], D [BH, Npad],
@@ -30,12 +43,17 @@ cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CU
 size_t sm100_backward_workspace(int BH, int N, int d);
 // byte offset of the fp32 dQ accumulator inside the workspace
 size_t sm100_backward_dq_offset(int BH, int N);
+// `stages` selects the launches (kStagePreprocess | kStageMain | kStageConvert
+// for the whole pass); each later stage reads what the earlier ones left in the
+// workspace.
+constexpr int kStagePreprocess = 1, kStageMain = 2, kStageConvert = 4, kStageAll = 7;
 // mq, mdo, mdq over Nq rows; mk, mv over Nk rows.
 // mdq: 3-D fp32 view {d, Nq, B*H} of the accumulator, box {32, 32, 1}, 128-byte swizzle
 cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                            const CUtensorMap& mdo, const CUtensorMap& mdq, const void* o,
                            const void* dout, const float* lse,
                            void* dq, void* dk, void* dv, void* workspace, int B, int H, int Hkv,
-                           int Nq, int Nk, int d, float scale, int causal, cudaStream_t st);
+                           int Nq, int Nk, int d, float scale, int causal, int stages,
+                           cudaStream_t st);
 
 }  // namespace fa

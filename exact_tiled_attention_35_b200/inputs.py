@@ -69,6 +69,38 @@ def make_inputs(B, H, N, d, dtype=torch.bfloat16, seed=0, qk_gain=1.0, with_do=F
     return tuple(out)
 
 
+E4M3_MAX = 448.0  # largest finite OCP FP8 E4M3 value
+
+
+def make_fp8_inputs(B, H, N, d, seed=0, qk_gain=1.0, Hkv=None, Nk=None):
+    """FP8 (e4m3) Q, K, V with one scale per tensor (CPU tensors).
+
+    Q, K, V are drawn as in ``make_inputs`` (same seed, same order), then each
+    tensor x is stored as e4m3(x / s) with s = amax(|x|) / 448, so its largest
+    value lands on the top of the e4m3 range; s is returned as the tensor's
+    descale (the stored values stand for s * stored).  With Hkv / Nk given, K and
+    V are drawn with those head count and length from seed + 100.
+    Returns (q8, k8, v8, q_descale, k_descale, v_descale)."""
+    q = make_inputs(B, H, N, d, dtype=torch.float32, seed=seed, qk_gain=qk_gain)[0]
+    if Hkv is None and Nk is None:
+        k, v = make_inputs(B, H, N, d, dtype=torch.float32, seed=seed, qk_gain=qk_gain)[1:3]
+    else:
+        k, v = make_inputs(B, Hkv or H, Nk or N, d, dtype=torch.float32, seed=seed + 100,
+                           qk_gain=qk_gain)[1:3]
+    out, scales = [], []
+    for x in (q, k, v):
+        s = float(x.abs().max()) / E4M3_MAX
+        s = s if s > 0 else 1.0
+        out.append((x / s).clamp(-E4M3_MAX, E4M3_MAX).to(torch.float8_e4m3fn))
+        scales.append(s)
+    return (*out, *scales)
+
+
+def fp8_values(x8, descale):
+    """The values an e4m3 tensor with a per-tensor descale stands for, float64 numpy."""
+    return x8.to(torch.float64).numpy() * float(descale)
+
+
 def sample_rows(N, count, seed, head):
     """Distinct query rows for one head: rows 0 and N-1 always, the rest uniform.
 

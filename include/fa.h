@@ -31,6 +31,15 @@
  * wait that runs out records FA_ERR_DEVICE_TIMEOUT in a device-side status
  * word instead of hanging, which fa_check_device_status reports.
  *
+ * Concurrency.  Calls on different streams may run at the same time.  Each
+ * forward launch draws its work items from one of 256 scheduler slots, taken
+ * round-robin, under an owner tag of its own; if two launches in flight ever
+ * meet on one slot, the later draws stop and FA_ERR_DEVICE_STATE is recorded
+ * rather than items being lost silently.  A forward launch captured into a CUDA
+ * graph keeps its slot and tag in every replay, so replays of one captured
+ * graph must not overlap each other on the GPU (replays in stream order are
+ * fine).
+ *
  * Limits.  d in {64, 128}; N >= 1 (any N: ragged tails are masked);
  * 1 <= B*H <= 65535*128; pointers 16-byte aligned; scale finite and > 0.
  */
@@ -50,7 +59,10 @@ typedef enum {
   FA_ERR_MISALIGNED = 3,     /* a pointer is not 16-byte aligned */
   FA_ERR_WORKSPACE = 4,      /* workspace missing or smaller than required */
   FA_ERR_CUDA = 5,           /* a CUDA runtime call or launch failed */
-  FA_ERR_DEVICE_TIMEOUT = 6  /* a kernel's bounded wait ran out */
+  FA_ERR_DEVICE_TIMEOUT = 6, /* a kernel's bounded wait ran out */
+  FA_ERR_DEVICE_STATE = 7    /* a kernel found device-side state it cannot trust
+                                (a scheduler slot held by another launch, a
+                                misaligned shared-memory base) and skipped work */
 } fa_status;
 
 /* Forward pass, bf16 storage, fp32 accumulation and statistics.
@@ -80,6 +92,23 @@ fa_status fa_forward_gqa(const void* q, const void* k, const void* v, void* o, f
 fa_status fa_forward_qk(const void* q, const void* k, const void* v, void* o, float* lse,
                         int B, int H, int Hkv, int Nq, int Nk, int d, float scale, int causal,
                         void* stream);
+
+/* FP8 forward (the FP8 support named in "Atención Flash-3" of the unite.ai page):
+ * Q, K, V stored as e4m3 (OCP FP8 E4M3, 1 byte per element) with one scale per
+ * tensor, so the values they stand for are q_descale * Q, k_descale * K and
+ * v_descale * V.  Both GEMMs run on the tensor cores in e4m3 with fp32
+ * accumulation: S = Q K^T, then P (the exponentials, at most 2^8) is rounded to
+ * e4m3 for P V.  Results as fa_forward_qk on the values they stand for:
+ *   O   = softmax(scale * q_descale * k_descale * Q K^T) (v_descale * V), bf16;
+ *   LSE = log sum_j exp(scale * q_descale * k_descale * q_i . k_j), fp32.
+ * q: [B,H,Nq,d], k, v: [B,Hkv,Nk,d] (e4m3); o: bf16 [B,H,Nq,d]; lse: fp32
+ * [B,H,Nq].  Grouped-query heads, lengths and causal mask as fa_forward_qk.
+ * The descales must be finite and > 0 (FA_ERR_INVALID_ARG otherwise); other
+ * errors as fa_forward.  The rounding of P to e4m3 (relative error up to 2^-4
+ * per element) makes O accurate to about 3 % rather than bf16's 0.5 %. */
+fa_status fa_forward_fp8(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                         int H, int Hkv, int Nq, int Nk, int d, float scale, float q_descale,
+                         float k_descale, float v_descale, int causal, void* stream);
 
 /* Forward pass with fp32 storage (q, k, v, o are float [B,H,N,d]); fp32
  * arithmetic on CUDA cores.  Same definition, same LSE convention. */
@@ -122,6 +151,27 @@ fa_status fa_backward_qk(const void* q, const void* k, const void* v, const void
                          void* workspace, size_t ws_bytes, int B, int H, int Hkv, int Nq, int Nk,
                          int d, float scale, int causal, void* stream);
 
+/* Stages of the bf16 backward pass, for callers that schedule or time them one
+ * by one (fa_backward runs all three in one call):
+ *   FA_STAGE_PREPROCESS  -LSE*log2(e) and -D_i = -sum_c dO[i,c] O[i,c] into the
+ *                        workspace, and a zeroed fp32 dQ accumulator there;
+ *   FA_STAGE_MAIN        P recomputed from Q, K and LSE; dK and dV written; the
+ *                        partial dQ = dS K of every key tile added into the
+ *                        accumulator;
+ *   FA_STAGE_DQ_CONVERT  dQ = scale * accumulator, rounded to bf16.
+ * Arguments as fa_backward_qk (Hkv = H and Nq = Nk for the square multi-head
+ * case) plus `stages`, a nonzero OR of the flags.  A later stage reads what an
+ * earlier one left in the workspace, so run them in this order, on one stream
+ * (or ordered by events), with the same arguments and workspace and nothing
+ * else writing the workspace in between. */
+#define FA_STAGE_PREPROCESS 1
+#define FA_STAGE_MAIN 2
+#define FA_STAGE_DQ_CONVERT 4
+fa_status fa_backward_stages(const void* q, const void* k, const void* v, const void* o,
+                             const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                             void* workspace, size_t ws_bytes, int B, int H, int Hkv, int Nq,
+                             int Nk, int d, float scale, int causal, int stages, void* stream);
+
 /* Backward pass with fp32 storage (all tensors float); CUDA-core arithmetic.
  * Workspace as for fa_backward. */
 fa_status fa_backward_fp32(const float* q, const float* k, const float* v, const float* o,
@@ -141,8 +191,10 @@ fa_status fa_backward_fp32(const float* q, const float* k, const float* v, const
  * fa_backward minus the workspace: the scratch lives in a fixed device array
  * inside the library (FA_BACKWARD_NOALLOC_MAX_BYTES), so this call allocates
  * nothing.  Shapes whose scratch (fa_backward_workspace_size) exceeds that
- * limit return FA_ERR_WORKSPACE.  The first call on a device looks up the
- * array's device address on that device (make it before any stream capture).
+ * limit return FA_ERR_WORKSPACE.  The first call in each CUDA context of a
+ * device (the first call on the device, and the first one after a
+ * cudaDeviceReset) looks up the array's device address there; make that call
+ * before any stream capture.
  * All calls share the one array and the kernels re-initialise what they read,
  * but two calls whose work overlaps on the GPU (different streams, no ordering
  * between them) race on it.  The pages have no counterpart to this entry
@@ -158,9 +210,22 @@ fa_status fa_backward_noalloc(const void* q, const void* k, const void* v, const
  * computation (the pages have no counterpart).  Returns FA_OK once launched. */
 fa_status fa_debug_wait_timeout(void* stream);
 
+/* Diagnostic: enqueues on `stream` a write that marks every slot of the forward
+ * pass's work-item scheduler as held by a launch that never finished, the state
+ * a crashed or abandoned launch could leave behind.  The next forward launch on
+ * the device then stops drawing work and records FA_ERR_DEVICE_STATE (outputs
+ * incomplete) instead of computing with the stale slot, and
+ * fa_check_device_status reports it and frees the slots.  Lets callers check
+ * that error path; the pages have no counterpart.  Returns FA_OK once enqueued. */
+fa_status fa_debug_hold_scheduler(void* stream);
+
 /* Synchronises `stream`, then reads and clears the current device's status
- * word.  FA_ERR_DEVICE_TIMEOUT if a kernel gave up a wait since the last call;
- * FA_ERR_CUDA if synchronisation failed; FA_OK otherwise. */
+ * word.  FA_ERR_DEVICE_TIMEOUT if a kernel gave up a wait since the last call,
+ * FA_ERR_DEVICE_STATE if a kernel skipped work because its device-side state was
+ * inconsistent (outputs written since the last call may be incomplete),
+ * FA_ERR_CUDA if synchronisation failed, FA_OK otherwise.  After reporting an
+ * error it also frees every slot of the forward pass's work-item scheduler, so
+ * call it while no other fa_* work is running on the device. */
 fa_status fa_check_device_status(void* stream);
 
 /* Text of the most recent CUDA error that an fa_* call on the calling thread

@@ -10,6 +10,7 @@ from .attention import (  # noqa: F401
     attention_fwd_gqa_ref,
     attention_fwd_ref,
     attention_rows_ref,
+    e4m3_p_rounding_bound,
     online_softmax_attention,
     safe_softmax,
     scores,

@@ -54,6 +54,7 @@ __all__ = [
     "online_softmax_attention",
     "attention_fwd_gqa_ref",
     "attention_bwd_gqa_ref",
+    "e4m3_p_rounding_bound",
 ]
 
 
@@ -278,3 +279,56 @@ def attention_bwd_gqa_ref(q, k, v, do, scale, causal):
     dk = dk_e.reshape(b_, hkv, group, n, d).sum(axis=2)
     dv = dv_e.reshape(b_, hkv, group, n, d).sum(axis=2)
     return dq, dk, dv
+
+
+# Facts of the OCP FP8 E4M3 format used by the FP8 forward ("Atención Flash-3",
+# item "Soporte para FP8", of the unite.ai page names FP8 support; the format
+# itself is not on the pages): 3 stored mantissa bits, so a value in the normal
+# range (>= 2^-6) is rounded to nearest with relative error at most 2^-4, and
+# below 2^-6 the spacing is 2^-9, so the absolute error is at most 2^-10.
+E4M3_REL = 2.0**-4
+E4M3_MIN_NORMAL = 2.0**-6
+E4M3_SUB_ABS = 2.0**-10
+
+
+def _e4m3_bound_from_scores(s, v):
+    m = np.max(s, axis=-1, keepdims=True)
+    m0 = np.where(np.isneginf(m), 0.0, m)
+    p = np.exp(s - m0)
+    l = np.sum(p, axis=-1, keepdims=True)
+    av = np.abs(_as64(v))
+    small = (p < E4M3_MIN_NORMAL) & ~np.isneginf(s)
+    num = E4M3_REL * np.matmul(p, av) + E4M3_SUB_ABS * np.matmul(small.astype(np.float64), av)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        return np.where(l > 0, num / np.where(l > 0, l, 1.0), 0.0)
+
+
+def e4m3_p_rounding_bound(q, k, v, scale, causal, rows=None):
+    """Worst-case |O_fp8 - O| per output element when the probabilities are
+    rounded to e4m3 before P V (the FP8 forward), everything else exact.
+
+    Reading (the pages give no error analysis): the kernel forms
+    p'_j = g * p_j with p_j = exp(S_ij - m_i) <= 1 and a factor g >= 1 (its
+    running maximum may trail the true one), rounds p'_j to e4m3 and divides the
+    sum of p'_j v_j by the unrounded sum g * l.  The rounding error of each p'_j
+    is at most 2^-4 p'_j, or 2^-10 when p'_j < 2^-6, so
+        |dO_ic| <= (2^-4 sum_j p_j |V_jc| + 2^-10 sum_{j: p_j < 2^-6} |V_jc|) / l
+    with l = sum_j p_j (g >= 1 only shrinks the second term).  Returns an array
+    of O's shape, or with ``rows`` (query indices per head, as for
+    ``attention_rows_ref``) the bound of those rows only, [B, H, R, d].
+    """
+    if rows is None:
+        return _e4m3_bound_from_scores(scores(q, k, scale, causal), v)
+    q, k, v = _as64(q), _as64(k), _as64(v)
+    b_, h_, n, d = q.shape
+    off = k.shape[2] - n
+    out = np.zeros((b_, h_, len(rows[0]), d))
+    for b in range(b_):
+        for h in range(h_):
+            for t, i in enumerate(rows[h]):
+                last = int(i) + off + 1 if causal else k.shape[2]
+                if last <= 0:
+                    continue
+                srow = scale * (k[b, h, :last] @ q[b, h, int(i)])
+                out[b, h, t] = _e4m3_bound_from_scores(srow[None, :], v[b, h, :last])[0]
+    return out

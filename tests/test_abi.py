@@ -124,3 +124,84 @@ def test_unequal_length_entry_points_reject_bad_arguments(lib):
         bad = list(ptrs)
         bad[i] = None
         assert b(*bad, ws, need, 1, 4, 2, 100, 300, 64, 0.125, 1, None) == INVALID
+
+
+def test_status_codes_have_strings(lib):
+    for code in range(8):
+        assert fa.status_string(code) != "unknown status", code
+
+
+def test_backward_stages_rejects_bad_arguments(lib):
+    f = lib.fa_backward_stages
+    ptrs = [P(0x10000 * (i + 1)) for i in range(9)]
+    ws = P(0x100000)
+    need = lib.fa_backward_workspace_size(1, 4, 100, 64)
+    for stages in (0, 8, -1, 15):
+        assert f(*ptrs, ws, need, 1, 4, 2, 100, 300, 64, 0.125, 1, stages, None) == INVALID
+    assert f(*ptrs, ws, need - 1, 1, 4, 2, 100, 300, 64, 0.125, 1, 2, None) == WORKSPACE
+    assert f(*ptrs, P(0x100004), need, 1, 4, 2, 100, 300, 64, 0.125, 1, 2, None) == MISALIGNED
+    assert f(*ptrs, ws, need, 1, 4, 3, 100, 300, 64, 0.125, 1, 7, None) == INVALID
+    for i in range(9):
+        bad = list(ptrs)
+        bad[i] = None
+        assert f(*bad, ws, need, 1, 4, 2, 100, 300, 64, 0.125, 1, 1, None) == INVALID
+
+
+def test_binding_checks_every_tensor_before_the_library():
+    # Shapes and dtypes of every argument are checked in the binding before any
+    # pointer reaches the library (CPU tensors: the checks run without a GPU and
+    # fail on the bad argument first).
+    import torch
+
+    B, H, N, d = 1, 2, 64, 64
+    q = torch.zeros(B, H, N, d, dtype=torch.bfloat16)
+    lse_ok = torch.zeros(B, H, N)
+    with pytest.raises(ValueError, match="lse"):
+        fa.forward(q, q, q, lse=torch.zeros(B, H, N + 1))
+    with pytest.raises(ValueError, match="lse"):
+        fa.forward(q, q, q, lse=torch.zeros(B, H, N, dtype=torch.float64))
+    with pytest.raises(ValueError, match="out"):
+        fa.forward(q, q, q, out=torch.zeros(B, H, N, d + 1, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="lse"):
+        fa.backward(q, q, q, q, q, torch.zeros(B, H, N - 1))
+    with pytest.raises(ValueError, match="dq"):
+        fa.backward(q, q, q, q, q, lse_ok, dq=torch.zeros(B, H, N, d))
+    with pytest.raises(ValueError, match="dk, dv"):
+        fa.backward(q, q, q, q, q, lse_ok, dv=torch.zeros(B, H, 2 * N, d, dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="q, o, do"):
+        fa.backward(q, q, q, q[:, :, :32].contiguous(), q, lse_ok)
+    with pytest.raises(ValueError, match="contiguous"):
+        fa.backward(q, q, q, q, q, lse_ok, dq=q.transpose(2, 3).contiguous().transpose(2, 3))
+    with pytest.raises(ValueError, match="lse"):
+        fa.backward_gqa(q, q[:, :1].contiguous(), q[:, :1].contiguous(), q, q, torch.zeros(B, H, N, 2))
+    with pytest.raises(ValueError, match="lse"):
+        fa.backward_noalloc(q, q, q, q, q, torch.zeros(B, H + 1, N))
+    with pytest.raises(ValueError, match="lse"):
+        fa.backward_stages(fa.STAGE_MAIN, q, q, q, q, q, torch.zeros(1), None, None, None, None)
+    with pytest.raises(ValueError, match="CUDA"):
+        fa.forward(q, q, q)  # well-formed, but on the host
+
+
+def test_noalloc_rejects_oversized_shapes_without_cuda(lib):
+    ptrs = [P(0x10000 * (i + 1)) for i in range(9)]
+    B, H, N, d = 4, 16, 4096, 128
+    assert lib.fa_backward_workspace_size(B, H, N, d) > 64 << 20
+    assert lib.fa_backward_noalloc(*ptrs, B, H, N, d, 0.088, 1, None) == WORKSPACE
+
+
+def test_fp8_forward_rejects_bad_arguments(lib):
+    f = lib.fa_forward_fp8
+    good = (1.0, 1.0, 1.0)
+    for qs, ks, vs in ((0.0, 1.0, 1.0), (1.0, -1.0, 1.0), (1.0, 1.0, float("nan")), (float("inf"), 1.0, 1.0),
+                       (1e-30, 1e-30, 1.0)):
+        assert f(*GOOD, 1, 2, 1, 16, 16, 64, 0.125, qs, ks, vs, 0, None) == INVALID, (qs, ks, vs)
+    assert f(*GOOD, 1, 2, 3, 16, 16, 64, 0.125, *good, 0, None) == INVALID  # Hkv does not divide H
+    assert f(*GOOD, 1, 2, 1, 0, 16, 64, 0.125, *good, 0, None) == INVALID
+    assert f(*GOOD, 1, 2, 1, 16, 16, 96, 0.125, *good, 0, None) == UNSUPPORTED
+    for i in range(5):
+        ptrs = list(GOOD)
+        ptrs[i] = None
+        assert f(*ptrs, 1, 2, 1, 16, 16, 64, 0.125, *good, 0, None) == INVALID
+    ptrs = list(GOOD)
+    ptrs[1] = P(0x20001)
+    assert f(*ptrs, 1, 2, 1, 16, 16, 64, 0.125, *good, 0, None) == MISALIGNED

@@ -33,3 +33,34 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     fa.check_device_status()
     o_ref, _ = attention_fwd_ref(to_f64(q.cpu()), to_f64(k.cpu()), to_f64(v.cpu()), 1 / math.sqrt(64), True)
     assert np.max(np.abs(to_f64(o) - o_ref)) < 1e-2
+
+
+FA_ERR_DEVICE_STATE = 7
+
+
+def test_stale_scheduler_slot_is_reported_not_used():
+    # A launch that never finished would leave its scheduler slot held.  The
+    # diagnostic marks every slot that way; the next forward must stop drawing
+    # work and report FA_ERR_DEVICE_STATE instead of handing out stale items,
+    # and after the status has been read (which frees the slots) the forward
+    # must be correct again.
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    lib = fa.load_library()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.fa_check_device_status(stream) == 0
+    q, k, v = (t.cuda() for t in make_inputs(2, 16, 2048, 64, seed=6))  # 256 items > one per SM
+    assert lib.fa_debug_hold_scheduler(stream) == 0
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full(q.shape[:3], float("nan"), device="cuda")
+    fa.forward(q, k, v, causal=True, out=o, lse=lse)
+    assert lib.fa_check_device_status(stream) == FA_ERR_DEVICE_STATE
+    assert bool(torch.isnan(o).any())  # items past each CTA's first were skipped, visibly
+    assert lib.fa_check_device_status(stream) == 0
+    o, lse = fa.forward(q, k, v, causal=True, out=o, lse=lse)
+    fa.check_device_status()
+    sl = (slice(1, 2), slice(15, 16))  # one head checked against the oracle
+    o_ref, _ = attention_fwd_ref(to_f64(q[sl].cpu()), to_f64(k[sl].cpu()), to_f64(v[sl].cpu()),
+                                 1 / math.sqrt(64), True)
+    assert not bool(torch.isnan(o).any())
+    assert np.max(np.abs(to_f64(o[sl]) - o_ref)) < 1e-2

@@ -485,3 +485,86 @@ def test_planted_top_left_alignment_is_caught():
     p = orc.safe_softmax(s)
     o_bad = np.einsum("bhij,bhjd->bhid", p, v)
     assert not np.allclose(o_bad, o_sq[:, :, nk - nq :], atol=1e-3)
+
+
+# ---------------------------------------------------------------- FP8 reading
+
+
+def _simulate_fp8_p(q, k, v, scale, causal, stale_log2=0.0):
+    """O with every probability rounded to e4m3 before P V, the way the FP8
+    forward does it: p' = g * exp(S - m) in float32 with g = 2^stale_log2 (a
+    running maximum that trails the true one), rounded to e4m3 by torch, summed
+    against V and divided by the unrounded g * l."""
+    s = orc.scores(q, k, scale, causal)
+    m = np.max(s, axis=-1, keepdims=True)
+    g = 2.0**stale_log2
+    p = (g * np.exp(s - m)).astype(np.float32)
+    p8 = torch.from_numpy(p).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    l = np.sum(p.astype(np.float64), axis=-1, keepdims=True)
+    return np.matmul(p8, v) / l
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("gain,stale", [(1.0, 0.0), (1.0, 5.3), (1.0, 8.0), (4.0, 0.0), (4.0, 7.5)])
+def test_e4m3_rounding_bound_holds_for_simulated_fp8(causal, gain, stale):
+    rng = np.random.default_rng(int(10 * gain + stale))
+    q, k, v = (rng.normal(size=(1, 2, 300, 64)) for _ in range(3))
+    q, k = q * gain, k * gain
+    o_ref, _ = orc.attention_fwd_ref(q, k, v, 0.125, causal)
+    o8 = _simulate_fp8_p(q, k, v, 0.125, causal, stale)
+    bound = orc.e4m3_p_rounding_bound(q, k, v, 0.125, causal)
+    err = np.abs(o8 - o_ref)
+    assert np.all(err <= bound * (1 + 1e-6) + 1e-12)
+    # the bound is a worst case, but not a vacuous one
+    assert np.max(err / np.maximum(bound, 1e-300)) > 0.05
+
+
+def test_e4m3_rounding_noise_is_what_the_tolerance_reading_says():
+    # rounding P to 3 mantissa bits adds relative noise of about 2^-3 / sqrt(12)
+    # times the mean of 2^e / p over a binade (0.72), i.e. ~2.6 % in O; the FP8
+    # parity bound allows rel-L2 <= 5e-2
+    rng = np.random.default_rng(3)
+    q, k, v = (rng.normal(size=(1, 4, 1024, 128)) for _ in range(3))
+    scale = 1 / math.sqrt(128)
+    for causal in (False, True):
+        o_ref, _ = orc.attention_fwd_ref(q, k, v, scale, causal)
+        o8 = _simulate_fp8_p(q, k, v, scale, causal)
+        rel = np.linalg.norm(o8 - o_ref) / np.linalg.norm(o_ref)
+        assert 0.01 < rel < 0.04, rel
+
+
+def test_e4m3_bound_rows_equal_full_bound():
+    rng = np.random.default_rng(4)
+    q, k, v = (rng.normal(size=(1, 2, 200, 32)) for _ in range(3))
+    full = orc.e4m3_p_rounding_bound(q, k, v, 0.2, True)
+    rows = [np.array([0, 17, 199]), np.array([3, 100, 150])]
+    part = orc.e4m3_p_rounding_bound(q, k, v, 0.2, True, rows=rows)
+    for h in range(2):
+        assert np.allclose(part[0, h], full[0, h, rows[h]], rtol=1e-12, atol=1e-15)
+
+
+def test_planted_fp8_slips_break_the_e4m3_bound():
+    # the bound admits e4m3 rounding of P and nothing else: a 10 % error in the
+    # score scale (a descale applied wrongly) or a running-maximum factor that is
+    # not divided out again must leave it
+    rng = np.random.default_rng(5)
+    q, k, v = (rng.normal(size=(1, 2, 256, 64)) for _ in range(3))
+    o_ref, _ = orc.attention_fwd_ref(q, k, v, 0.125, False)
+    bound = orc.e4m3_p_rounding_bound(q, k, v, 0.125, False)
+    wrong_scale = _simulate_fp8_p(q, k * 1.1, v, 0.125, False)
+    assert np.any(np.abs(wrong_scale - o_ref) > bound)
+    kept_factor = _simulate_fp8_p(q, k, v, 0.125, False, stale_log2=1.0) * 2.0
+    assert np.any(np.abs(kept_factor - o_ref) > bound)
+
+
+def test_fp8_inputs_recipe():
+    from exact_tiled_attention_35_b200.inputs import fp8_values, make_fp8_inputs, make_inputs
+
+    q8, k8, v8, qs, ks, vs = make_fp8_inputs(1, 2, 100, 64, seed=3)
+    q32 = make_inputs(1, 2, 100, 64, dtype=torch.float32, seed=3)[0].double().numpy()
+    for x8, s in ((q8, qs), (k8, ks), (v8, vs)):
+        assert x8.dtype == torch.float8_e4m3fn
+        assert float(x8.float().abs().max()) == 448.0  # amax lands on the top of the range
+    # decoded values are within e4m3 rounding of the drawn ones
+    err = np.abs(fp8_values(q8, qs) - q32)
+    assert np.all(err <= 2.0**-4 * np.abs(q32) + 2.0**-10 * qs + 1e-12)

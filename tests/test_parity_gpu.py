@@ -1,17 +1,10 @@
 """Parity of the CUDA path (through the C ABI) with the fp64 oracle, on the same
-seeded inputs.  GPU only.
+seeded inputs.  GPU only.  Bounds and error measures: tests/parity.py (bf16
+forward O within 1e-2 of the oracle before the output's bf16 rounding, rel-L2
+<= 5e-3, LSE max-abs <= 1e-2; dQ/dK/dV rel-L2 <= 2e-2).  Outputs are filled with
+NaN before every call, so a row or gradient the kernels never write fails.
 
-Tolerances (from the method's task statement): bf16 forward O max-abs <= 1e-2
-and rel-L2 <= 5e-3; dQ/dK/dV rel-L2 <= 2e-2.  LSE: max-abs <= 1e-2 (reading:
-the statement names no LSE tolerance; the forward's absolute bound is reused).
-The fp32-storage path is held to the same forward bounds.
-
-Reading of the max-abs bound for bf16 outputs: O is stored in bf16, whose
-spacing is 2^-5 for |O| in [4, 8), so even the exact result rounded to bf16 can
-sit 0.0156 from the fp64 value.  The bound is applied element by element as
-1e-2 plus half the bf16 spacing at the reference value (the storage rounding no
-implementation with bf16 output can avoid); it equals 1e-2 plus at most 2^-9
-of |O| and changes nothing where |O| < 2.
+The five workloads at their full sizes are checked in test_parity_report_gpu.py.
 """
 
 import math
@@ -21,34 +14,11 @@ import pytest
 import torch
 
 import exact_tiled_attention_35_b200 as fa
-from exact_tiled_attention_35_b200.inputs import WORKLOADS, make_inputs, sample_rows, to_f64
-from oracle import attention_bwd_ref, attention_fwd_ref, attention_rows_ref
+from exact_tiled_attention_35_b200.inputs import make_inputs, to_f64
+from oracle import attention_bwd_ref, attention_fwd_ref
+from parity import O_MAXABS, check_bwd, check_fwd, max_abs, rel_l2
 
 pytestmark = pytest.mark.gpu
-
-O_MAXABS, O_RELL2, LSE_MAXABS, GRAD_RELL2 = 1e-2, 5e-3, 1e-2, 2e-2
-
-
-def rel_l2(x, ref):
-    return float(np.linalg.norm((x - ref).ravel()) / np.linalg.norm(ref.ravel()))
-
-
-def max_abs(x, ref):
-    return float(np.max(np.abs(x - ref)))
-
-
-def bf16_half_spacing(x):
-    """Half the distance between adjacent bf16 values at |x| (8-bit significand)."""
-    e = np.floor(np.log2(np.maximum(np.abs(x), 2.0**-126)))
-    return 0.5 * 2.0 ** (e - 7)
-
-
-def check_fwd(o, lse, o_ref, lse_ref, what, bf16_out=True):
-    assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse)), what
-    ma, rl, ml = max_abs(o, o_ref), rel_l2(o, o_ref), max_abs(lse, lse_ref)
-    bound = O_MAXABS + (bf16_half_spacing(o_ref) if bf16_out else 0.0)
-    excess = float(np.max(np.abs(o - o_ref) - bound))
-    assert excess <= 0 and rl <= O_RELL2 and ml <= LSE_MAXABS, (what, ma, excess, rl, ml)
 
 
 def run_fwd(B, H, N, d, causal, dtype=torch.bfloat16, seed=0, gain=1.0):
@@ -87,47 +57,11 @@ def test_forward_several_heads_and_batches(seed):
     check_fwd(o, lse, o_ref, lse_ref, seed)
 
 
-def test_forward_fp32_small_config():
-    w = WORKLOADS["fwd_b1h1n256d64_fp32"]
-    (q, k, v), o, lse = run_fwd(w.B, w.H, w.N, w.d, w.causal, dtype=torch.float32)
-    o_ref, lse_ref = attention_fwd_ref(to_f64(q), to_f64(k), to_f64(v), w.scale, w.causal)
-    check_fwd(o, lse, o_ref, lse_ref, w.name, bf16_out=False)
-    # fp32 storage: far inside the bound
-    assert max_abs(o, o_ref) < 1e-4
-
-
 @pytest.mark.parametrize("N,causal", [(256, True), (333, False)])
 def test_forward_fp32_sweep(N, causal):
     (q, k, v), o, lse = run_fwd(2, 2, N, 128, causal, dtype=torch.float32, seed=5)
     o_ref, lse_ref = attention_fwd_ref(to_f64(q), to_f64(k), to_f64(v), 1 / math.sqrt(128), causal)
     check_fwd(o, lse, o_ref, lse_ref, N, bf16_out=False)
-
-
-def test_forward_gpt2_like_config_full():
-    w = WORKLOADS["fwd_b4h16n1024d64"]
-    (q, k, v), o, lse = run_fwd(w.B, w.H, w.N, w.d, w.causal)
-    o_ref, lse_ref = attention_fwd_ref(to_f64(q), to_f64(k), to_f64(v), w.scale, w.causal)
-    check_fwd(o, lse, o_ref, lse_ref, w.name)
-
-
-def _sampled_check(w, rows_per_head, seed=0):
-    (q, k, v), o, lse = run_fwd(w.B, w.H, w.N, w.d, w.causal, seed=seed, gain=w.qk_gain)
-    rows = [sample_rows(w.N, rows_per_head, seed, h) for h in range(w.H)]
-    o_ref, lse_ref = attention_rows_ref(to_f64(q), to_f64(k), to_f64(v), rows, w.scale, w.causal)
-    o_s = np.stack([o[:, h, rows[h]] for h in range(w.H)], axis=1)
-    l_s = np.stack([lse[:, h, rows[h]] for h in range(w.H)], axis=1)
-    check_fwd(o_s, l_s, o_ref, lse_ref, w.name)
-    return o, lse
-
-
-def test_forward_causal_4096_d128_sampled():
-    w = WORKLOADS["fwd_b2h32n4096d128_causal"]
-    _sampled_check(w, 64)
-
-
-def test_forward_long_context_stress_sampled():
-    w = WORKLOADS["fwd_b1h8n32768d128_causal_x4"]
-    _sampled_check(w, w.sampled_rows)
 
 
 def test_forward_is_deterministic():
@@ -196,19 +130,10 @@ def run_bwd(B, H, N, d, causal, dtype=torch.bfloat16, seed=0):
     q, k, v, do = make_inputs(B, H, N, d, dtype=dtype, seed=seed, with_do=True)
     qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
     o, lse = fa.forward(qd, kd, vd, causal=causal)
-    dq, dk, dv = fa.backward(qd, kd, vd, o, dod, lse, causal=causal)
+    dq, dk, dv = (torch.full_like(t, float("nan")) for t in (qd, kd, vd))
+    fa.backward(qd, kd, vd, o, dod, lse, causal=causal, dq=dq, dk=dk, dv=dv)
     fa.check_device_status()
     return (q, k, v, do), tuple(to_f64(x) for x in (dq, dk, dv))
-
-
-def check_bwd(got, ref, what):
-    for name, g, r in zip(("dq", "dk", "dv"), got, ref):
-        assert np.all(np.isfinite(g)), (what, name)
-        if np.linalg.norm(r) < 1e-12:  # e.g. N == 1: dQ = dK = 0 exactly
-            assert max_abs(g, r) <= 1e-3, (what, name)
-            continue
-        e = rel_l2(g, r)
-        assert e <= GRAD_RELL2, (what, name, e)
 
 
 @pytest.mark.parametrize("d", [64, 128])
@@ -225,15 +150,6 @@ def test_backward_fp32_storage():
     ref = attention_bwd_ref(to_f64(q), to_f64(k), to_f64(v), to_f64(do), 1 / 8.0, True)
     for g, r in zip(got, ref):
         assert rel_l2(g, r) < 1e-5
-
-
-def test_backward_config_2048_d128_causal_heads():
-    w = WORKLOADS["fwdbwd_b2h16n2048d128_causal"]
-    (q, k, v, do), got = run_bwd(w.B, w.H, w.N, w.d, w.causal)
-    for b, h in [(0, 0), (0, 7), (1, 3), (1, 15)]:
-        sl = lambda x: to_f64(x)[b : b + 1, h : h + 1]
-        ref = attention_bwd_ref(sl(q), sl(k), sl(v), sl(do), w.scale, w.causal)
-        check_bwd(tuple(g[b : b + 1, h : h + 1] for g in got), ref, (b, h))
 
 
 @pytest.mark.parametrize("B,H,Hkv,N,d,causal", [(2, 16, 16, 2048, 128, True), (2, 32, 32, 4096, 128, True),
@@ -275,7 +191,8 @@ def test_gqa_forward_and_backward(H, Hkv, N, causal, d):
     _, k, v = make_inputs(1, Hkv, N, d, seed=7 + Hkv)
     qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
     o, lse = fa.forward_gqa(qd, kd, vd, causal=causal)
-    dq, dk, dv = fa.backward_gqa(qd, kd, vd, o, dod, lse, causal=causal)
+    dq, dk, dv = (torch.full_like(t, float("nan")) for t in (qd, kd, vd))
+    fa.backward_gqa(qd, kd, vd, o, dod, lse, causal=causal, dq=dq, dk=dk, dv=dv)
     fa.check_device_status()
     scale = 1 / math.sqrt(d)
     o_ref, lse_ref = attention_fwd_gqa_ref(to_f64(q), to_f64(k), to_f64(v), scale, causal)
@@ -318,7 +235,10 @@ def test_forward_unequal_lengths(Nq, Nk, causal, d):
     from oracle import attention_fwd_gqa_ref
 
     q, k, v, _ = _qk_inputs(1, 4, 2, Nq, Nk, d, seed=Nq + Nk)
-    o, lse = fa.forward_qk(*(t.cuda() for t in (q, k, v)), causal=causal)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o = torch.full_like(qd, float("nan"))
+    lse = torch.full(qd.shape[:3], float("nan"), device="cuda")
+    fa.forward_qk(qd, kd, vd, causal=causal, out=o, lse=lse)
     fa.check_device_status()
     o_ref, lse_ref = attention_fwd_gqa_ref(to_f64(q), to_f64(k), to_f64(v), 1 / math.sqrt(d), causal)
     _check_fwd_with_empty_rows(to_f64(o), to_f64(lse), o_ref, lse_ref, (Nq, Nk, causal, d))
@@ -333,7 +253,8 @@ def test_backward_unequal_lengths(Nq, Nk, causal, d):
     q, k, v, do = _qk_inputs(1, 4, 2, Nq, Nk, d, seed=7 * Nq + Nk)
     qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
     o, lse = fa.forward_qk(qd, kd, vd, causal=causal)
-    dq, dk, dv = fa.backward_qk(qd, kd, vd, o, dod, lse, causal=causal)
+    dq, dk, dv = (torch.full_like(t, float("nan")) for t in (qd, kd, vd))
+    fa.backward_qk(qd, kd, vd, o, dod, lse, causal=causal, dq=dq, dk=dk, dv=dv)
     fa.check_device_status()
     ref = attention_bwd_gqa_ref(to_f64(q), to_f64(k), to_f64(v), to_f64(do), 1 / math.sqrt(d), causal)
     check_bwd(tuple(to_f64(x) for x in (dq, dk, dv)), ref, (Nq, Nk, causal, d))
