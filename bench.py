@@ -422,8 +422,35 @@ def run_ours(args, w, world, rank, local):
             else "fallback bf16 burst (no MEASURED_PEAKS.json)",
             "traffic": profiled_traffic(dom["kernel"], w.name)}
 
-    # the other workloads, forward alone, each timed the same way
+    # the deterministic backward on the same workload (separate dQ pass), its
+    # three stages timed the same way
     extras = {}
+    if w.backward and not args.skip_extras:
+        det = fa.STAGE_DETERMINISTIC
+        ev2 = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+        for _ in range(args.warmup):
+            flush.zero_()
+            for stage in (fa.STAGE_PREPROCESS, fa.STAGE_MAIN, fa.STAGE_DQ_CONVERT):
+                codes.append(prob.backward(stage | det))
+        torch.cuda.synchronize()
+        for e in ev2:
+            flush.zero_()
+            e[0].record()
+            for s_i, stage in enumerate((fa.STAGE_PREPROCESS, fa.STAGE_MAIN, fa.STAGE_DQ_CONVERT)):
+                codes.append(prob.backward(stage | det))
+                e[s_i + 1].record()
+        torch.cuda.synchronize()
+        _check_codes(codes, fa)
+        fa.check_device_status()
+        seg2 = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in ev2) for j in range(3)]
+        tot = max_over_ranks(sum(seg2), world)
+        extras["backward_deterministic"] = {
+            "workload": w.name, "ms": tot, "tflops": bwd_flops / (tot * 1e-3) / 1e12,
+            "breakdown_ms": {"preprocess": seg2[0], "main_dk_dv": seg2[1], "dq_pass": seg2[2]},
+            "note": "fa_backward_deterministic's three launches; TFLOP/s on the same algorithmic "
+                    "10*B*H*N^2*d/2 as the single-pass backward (it executes 14 instead of 10)"}
+
+    # the other workloads, forward alone, each timed the same way
     if not args.skip_extras:
         for key, name in (("forward_target", FWD_TARGET_WORKLOAD), ("short_seq_forward", "fwd_b4h16n1024d64"),
                           ("long_context_forward", "fwd_b1h8n32768d128_causal_x4")):

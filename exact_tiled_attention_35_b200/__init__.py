@@ -18,7 +18,8 @@ import os
 import torch
 
 __all__ = ["forward", "forward_fp8", "backward", "forward_gqa", "backward_gqa", "forward_qk", "backward_qk",
-           "backward_stages", "backward_noalloc", "STAGE_PREPROCESS", "STAGE_MAIN", "STAGE_DQ_CONVERT", "FAError", "library_path", "load_library", "check_device_status",
+           "backward_stages", "backward_deterministic", "backward_noalloc", "STAGE_PREPROCESS",
+           "STAGE_MAIN", "STAGE_DQ_CONVERT", "STAGE_DETERMINISTIC", "FAError", "library_path", "load_library", "check_device_status",
            "workspace_size", "SYMBOLS"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -38,6 +39,7 @@ SYMBOLS = {
     "fa_backward_qk": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_fp32": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_stages": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "fa_backward_deterministic": (_I, [_P] * 9 + [_P, _Z, _I, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_backward_noalloc": (_I, [_P] * 9 + [_I, _I, _I, _I, _F, _I, _P]),
     "fa_debug_wait_timeout": (_I, [_P]),
     "fa_debug_hold_scheduler": (_I, [_P]),
@@ -299,7 +301,23 @@ def backward_qk(q, k, v, o, do, lse, causal=False, scale=None, dq=None, dk=None,
     return dq, dk, dv
 
 
-STAGE_PREPROCESS, STAGE_MAIN, STAGE_DQ_CONVERT = 1, 2, 4
+STAGE_PREPROCESS, STAGE_MAIN, STAGE_DQ_CONVERT, STAGE_DETERMINISTIC = 1, 2, 4, 8
+
+
+def backward_deterministic(q, k, v, o, do, lse, causal=False, scale=None, dq=None, dk=None, dv=None,
+                           workspace=None):
+    """dQ [B,H,Nq,d], dK and dV [B,Hkv,Nk,d] via fa_backward_deterministic (bf16):
+    the same results as backward_qk, reproducible bit for bit (dQ by a separate
+    pass over the key tiles in a fixed order)."""
+    B, H, Hkv, Nq, Nk, d, dq, dk, dv = _bwd_tensors(q, k, v, o, do, lse, dq, dk, dv, torch.bfloat16)
+    scale = _scale(scale, d)
+    lib = load_library()
+    workspace = _workspace(workspace, int(lib.fa_backward_workspace_size(B, H, Nq, d)), q.device)
+    _check(lib.fa_backward_deterministic(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                                         _ptr(dk), _ptr(dv), _ptr(workspace), _nbytes(workspace), B, H, Hkv,
+                                         Nq, Nk, d, scale, int(bool(causal)), _stream(q)),
+           "fa_backward_deterministic")
+    return dq, dk, dv
 
 
 def backward_stages(stages, q, k, v, o, do, lse, dq, dk, dv, workspace, causal=False, scale=None):

@@ -18,7 +18,7 @@
 namespace fa {
 
 static_assert(FA_STAGE_PREPROCESS == kStagePreprocess && FA_STAGE_MAIN == kStageMain &&
-                  FA_STAGE_DQ_CONVERT == kStageConvert,
+                  FA_STAGE_DQ_CONVERT == kStageConvert && FA_STAGE_DETERMINISTIC == kStageDeterministic,
               "stage flags of the header and the kernels differ");
 
 // the device status word g_device_status is defined in fa_device.cuh
@@ -210,7 +210,8 @@ fa_status backward_entry(const void* q, const void* k, const void* v, const void
   if (s != FA_OK) return s;
   if ((s = check_shape(B, H, Nk, d, scale)) != FA_OK) return s;
   if (Hkv <= 0 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
-  if (stages <= 0 || stages > kStageAll) return FA_ERR_INVALID_ARG;
+  if ((stages & kStageAll) == 0 || (stages & ~(kStageAll | kStageDeterministic)) != 0)
+    return FA_ERR_INVALID_ARG;
   if ((s = check_ptrs({q, k, v, o, dout, lse, dq, dk, dv})) != FA_OK) return s;
   if (workspace == nullptr || ws_bytes < ws_bytes_for(B, H, Nq, d)) return FA_ERR_WORKSPACE;
   if (!aligned16(workspace)) return FA_ERR_MISALIGNED;
@@ -298,6 +299,14 @@ fa_status fa_backward_qk(const void* q, const void* k, const void* v, const void
                          int d, float scale, int causal, void* stream) {
   return backward_entry(q, k, v, o, dout, lse, dq, dk, dv, workspace, ws_bytes, B, H, Hkv, Nq, Nk, d,
                         scale, causal, kStageAll, stream);
+}
+
+fa_status fa_backward_deterministic(const void* q, const void* k, const void* v, const void* o,
+                                   const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                   void* workspace, size_t ws_bytes, int B, int H, int Hkv, int Nq,
+                                   int Nk, int d, float scale, int causal, void* stream) {
+  return backward_entry(q, k, v, o, dout, lse, dq, dk, dv, workspace, ws_bytes, B, H, Hkv, Nq, Nk, d,
+                        scale, causal, kStageAll | kStageDeterministic, stream);
 }
 
 fa_status fa_backward_stages(const void* q, const void* k, const void* v, const void* o,

@@ -157,7 +157,10 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
-template <int D>
+// kDQ: also form the partial dQ = dS K of every query tile and add it into the
+// fp32 accumulator (the single-pass backward); without it the kernel computes
+// dK and dV only and dQ comes from dq_kernel.
+template <int D, bool kDQ>
 __global__ void __launch_bounds__(NTHREADS, 1)
     main_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                 const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
@@ -346,13 +349,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         ok = mbar_wait(&bars->ds_full, it & 1, 38);
         if (!ok) break;
         tc_fence_after();
-        // dQ_part = dS K  (queries x d), K = 128 keys; written over dP^T
-        const uint64_t dmn = opaque(d0) + kToMn;
+        if constexpr (kDQ) {
+          // dQ_part = dS K  (queries x d), K = 128 keys; written over dP^T
+          const uint64_t dmn = opaque(d0) + kToMn;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ss(tmem + C::T_DP, sdesc_at(dmn, C::OFF_DS + kk * 2048), sdesc_at(dmn, C::OFF_K + kk * 2048),
-                 C::IDESC_DQ, kk > 0);
-        mma_commit(&bars->dq_full);
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_ss(tmem + C::T_DP, sdesc_at(dmn, C::OFF_DS + kk * 2048), sdesc_at(dmn, C::OFF_K + kk * 2048),
+                   C::IDESC_DQ, kk > 0);
+          mma_commit(&bars->dq_full);
+        }
         // dK += dS^T Q  (keys x d), K = 128 queries
         const uint64_t dq_mn = q_desc(it) + kToMn, dds = opaque(d0);
 #pragma unroll
@@ -364,7 +369,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mma_commit(&bars->ds_free);
         mma_commit(&bars->q_empty[st]);
         if (more) {
-          ok = mbar_wait(&bars->dq_empty, it & 1, 37);
+          // dP^T(i+1) overwrites the columns dQ(i) was drained from; without dQ
+          // the compute warps have read dP^T(i) before they published dS(i)
+          if constexpr (kDQ) ok = mbar_wait(&bars->dq_empty, it & 1, 37);
           if (ok) ok = mbar_wait(&bars->do_full, (it + 1) & 1, 49);
           if (!ok) break;
           tc_fence_after();
@@ -507,6 +514,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
       }
     }
+  } else if constexpr (!kDQ) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsReduce));
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsReduce));
     // dQ reduce warps 8-11: warp w drains query rows 32*(w%4) .. +31 of each
@@ -563,10 +572,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   }
 }
 
-// -D, -LSE*log2(e) (padded; the main kernel adds them) and a zeroed dQ
-// accumulator.  A row of O and dO is D/8 lanes' worth of 16-byte loads, so a
-// warp covers 256/D rows at once; every access is a 16-byte vector.
-template <int D>
+// -D, -LSE*log2(e) (padded; the main kernel adds them) and, for the single-pass
+// backward, a zeroed dQ accumulator.  A row of O and dO is D/8 lanes' worth of
+// 16-byte loads, so a warp covers 256/D rows at once; every access is a 16-byte
+// vector.  (Four rows per lane with all loads issued first measured slower: the
+// 64-bit row arithmetic per pass and the lower occupancy outweighed the extra
+// loads in flight.)
+template <int D, bool kZeroAcc>
 __global__ void __launch_bounds__(256) preprocess_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dout,
                                                          const float* __restrict__ lse,
@@ -578,6 +590,7 @@ __global__ void __launch_bounds__(256) preprocess_kernel(const __nv_bfloat16* __
   constexpr int RPW = 32 / L;       // rows per warp
   const int lane = threadIdx.x % 32;
   const long long gr = ((long long)blockIdx.x * 8 + threadIdx.x / 32) * RPW + lane / L;
+  // BH * Npad is a multiple of 128, hence of RPW: whole warps leave here together
   if (gr >= (long long)BH * Npad) return;
   const int bh = (int)(gr / Npad), row = (int)(gr % Npad);
   const int c = (lane % L) * 8;
@@ -594,9 +607,11 @@ __global__ void __launch_bounds__(256) preprocess_kernel(const __nv_bfloat16* __
       acc = fmaf(af.x, gf.x, acc);
       acc = fmaf(af.y, gf.y, acc);
     }
-    float4* z = reinterpret_cast<float4*>(dq_acc + off);
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if constexpr (kZeroAcc) {
+      float4* z = reinterpret_cast<float4*>(dq_acc + off);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
   // the L lanes of a row are consecutive and L-aligned: reduce within them
 #pragma unroll
@@ -614,23 +629,405 @@ __global__ void __launch_bounds__(256) preprocess_kernel(const __nv_bfloat16* __
   }
 }
 
-// dQ = scale * accumulator in bf16: eight values per thread (two 16-byte loads,
-// one 16-byte store).
+// dQ = scale * accumulator in bf16: sixteen values per thread (four 16-byte
+// loads issued together, two 16-byte stores).
 __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict__ acc,
-                                                         __nv_bfloat16* __restrict__ dq, long long n8,
+                                                         __nv_bfloat16* __restrict__ dq, long long n16,
                                                          float scale) {
-  for (long long idx = (long long)blockIdx.x * 256 + threadIdx.x; idx < n8;
+  for (long long idx = (long long)blockIdx.x * 256 + threadIdx.x; idx < n16;
        idx += (long long)gridDim.x * 256) {
-    const float4 a = reinterpret_cast<const float4*>(acc)[2 * idx];
-    const float4 b = reinterpret_cast<const float4*>(acc)[2 * idx + 1];
-    uint4 w;
-    w.x = pack_bf16x2(a.x * scale, a.y * scale);
-    w.y = pack_bf16x2(a.z * scale, a.w * scale);
-    w.z = pack_bf16x2(b.x * scale, b.y * scale);
-    w.w = pack_bf16x2(b.z * scale, b.w * scale);
-    reinterpret_cast<uint4*>(dq)[idx] = w;
+    const float4* src = reinterpret_cast<const float4*>(acc) + 4 * idx;
+    float4 v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = __ldcs(src + k);  // read once: streaming
+    uint4 w[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      w[k].x = pack_bf16x2(v[2 * k].x * scale, v[2 * k].y * scale);
+      w[k].y = pack_bf16x2(v[2 * k].z * scale, v[2 * k].w * scale);
+      w[k].z = pack_bf16x2(v[2 * k + 1].x * scale, v[2 * k + 1].y * scale);
+      w[k].w = pack_bf16x2(v[2 * k + 1].z * scale, v[2 * k + 1].w * scale);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(dq) + 2 * idx;
+    dst[0] = w[0];
+    dst[1] = w[1];
   }
 }
+
+// ---------------------------------------------------------------- dQ pass
+//
+// The deterministic dQ: one CTA per (128-row query tile, query head) walks the
+// key tiles the tile sees in a fixed order and accumulates
+//   dQ = scale * sum_j dS_j K_j,  dS_j = P_j * (dP_j - D),  P_j = exp2(S_j c - LSE2),
+//   S_j = Q K_j^T,  dP_j = dO V_j^T
+// in tensor memory, so no partial sums cross CTAs and the result does not
+// depend on scheduling.  Q and dO stay in tensor memory for the whole pass
+// (copied in once from their TMA tiles), which makes all three GEMMs of a key
+// tile tensor-memory-A forms that read only K_j or V_j from shared memory.
+//
+// CTA layout (384 threads, registers rebalanced as in the forward):
+//   warps 0-7  dS (thread = query row = tensor-memory lane; two warps per lane
+//              quarter, one per half of the key columns) and the dQ epilogue
+//   warp  8    TMA producer: Q, dO and the LSE2 / D rows once, then K_j, V_j
+//   warp  9    tensor-memory allocator and MMA issuer (warps 10-11 idle)
+// Tensor memory: Q (bf16, D/2 columns) at 0, dO at D/2, S at D, dP at D + 128
+// (dS in bf16 written over the first half of each warp's own dP columns), dQ at
+// D + 256.
+namespace dqp {
+
+constexpr int NTHREADS = 384;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kRegsCompute = 208;
+constexpr int kRegsControl = 88;
+static_assert(128 * (2 * kRegsCompute + kRegsControl) <= NTHREADS * 168,
+              "register split exceeds the launch allocation");
+
+template <int D>
+struct Cfg {
+  static constexpr int TILE = BN * D * 2;
+  static constexpr int CHUNK = BN * 128;
+  static constexpr int NSLOT = D == 128 ? 5 : 8;  // K/V ring slots
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_DO = TILE;
+  static constexpr int OFF_RING = 2 * TILE;
+  static constexpr int OFF_VEC = OFF_RING + NSLOT * TILE;  // LSE2 row values, then -D
+  static constexpr int OFF_BAR = OFF_VEC + 2 * BM * 4;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t T_Q = 0, T_DO = D / 2, T_S = D, T_DP = D + 128, T_DQ = D + 256;
+  static constexpr uint32_t IDESC_S = idesc_bf16(BM, BN, 0, 0);   // Q (tmem) x K (K-major)
+  static constexpr uint32_t IDESC_DQ = idesc_bf16(BM, D, 0, 1);   // dS (tmem) x K (MN-major)
+  static_assert(T_DQ + D <= TMEM_COLS, "tensor memory over budget");
+  static_assert(SMEM_BYTES <= 232448, "shared memory over the per-block limit");
+};
+
+struct Params {
+  __nv_bfloat16* dq;
+  const float* lse2;  // [BH, Npad]  -LSE * log2(e), -inf on padding rows
+  const float* dsum;  // [BH, Npad]  -D
+  int BH, H, G, Nq, Nk, off, Npad, nq, chunk, causal;
+  float scale, scale_log2;
+};
+
+struct Bars {
+  uint64_t q_full;   // Q, dO tiles and the row vectors
+  uint64_t q_ready;  // Q and dO copied into tensor memory
+  uint64_t kv_full[8];
+  uint64_t kv_empty[8];
+  uint64_t s_full, s_free, dp_full, ds_full, dq_done, drain;
+  uint32_t tmem_base;
+};
+
+// key tiles the query tile starting at row q0 sees (as the forward's tiles_for)
+__device__ __forceinline__ int key_tiles(int q0, const Params& p) {
+  const int nkv = (p.Nk + BN - 1) / BN;
+  if (!p.causal) return nkv;
+  const int kmax = min(q0 + BM - 1, p.Nq - 1) + p.off;
+  return kmax < 0 ? 0 : min(nkv, kmax / BN + 1);
+}
+
+template <int D>
+__global__ void __launch_bounds__(NTHREADS, 1)
+    dq_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+              const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
+              const Params p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  float* sVec = reinterpret_cast<float*>(smem + C::OFF_VEC);
+  Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  // CTA -> (query head, query tile): heads in L2-sized chunks, within a chunk
+  // the tiles that see the most keys first
+  const int per_chunk = p.chunk * p.nq;
+  const int chunk_id = blockIdx.x / per_chunk, w_in = blockIdx.x - chunk_id * per_chunk;
+  const int h0 = chunk_id * p.chunk, hn = min(p.chunk, p.BH - h0);
+  const int rank = w_in / hn;
+  const int bh = h0 + (w_in - rank * hn);
+  const int i = p.causal ? p.nq - 1 - rank : rank;  // query tile
+  const int bkv = (bh / p.H) * (p.H / p.G) + (bh % p.H) / p.G;
+  const int n = key_tiles(i * BM, p);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_ready, 256);
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(&bars->kv_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, 256);
+    mbar_init(&bars->dp_full, 1);
+    mbar_init(&bars->ds_full, 256);
+    mbar_init(&bars->dq_done, 1);
+    mbar_init(&bars->drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    tma_prefetch_desc(&mq);
+    tma_prefetch_desc(&mk);
+    tma_prefetch_desc(&mv);
+    tma_prefetch_desc(&mdo);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp >= 8) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
+    if (warp == kProducerWarp && lane == 0) {
+      mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE + 2 * BM * 4);
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d(smem + C::OFF_Q + c * C::CHUNK, &mq, &bars->q_full, c * 64, i * BM, bh);
+        tma_load_3d(smem + C::OFF_DO + c * C::CHUNK, &mdo, &bars->q_full, c * 64, i * BM, bh);
+      }
+      const size_t voff = (size_t)bh * p.Npad + (size_t)i * BM;
+      bulk_load(sVec, p.lse2 + voff, BM * 4, &bars->q_full);
+      bulk_load(sVec + BM, p.dsum + voff, BM * 4, &bars->q_full);
+      bool ok = true;
+      // ring sequence K_0, V_0, K_1, V_1, ...
+      for (int s2 = 0; s2 < 2 * n && ok; ++s2) {
+        const int slot = s2 % C::NSLOT, round = s2 / C::NSLOT;
+        if (round > 0) ok = mbar_wait(&bars->kv_empty[slot], (round - 1) & 1, 60);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bars->kv_full[slot], C::TILE);
+        const CUtensorMap* m = (s2 & 1) ? &mv : &mk;
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(smem + C::OFF_RING + slot * C::TILE + c * C::CHUNK, m, &bars->kv_full[slot], c * 64,
+                      (s2 >> 1) * BN, bkv);
+      }
+      // no copy into this CTA's shared memory may be in flight at exit
+      mbar_wait(&bars->q_full, 0, 61);
+      const int issued = ok ? 2 * n : 0;
+      for (int slot = 0; slot < C::NSLOT && slot < issued; ++slot) {
+        const int last = slot + ((issued - 1 - slot) / C::NSLOT) * C::NSLOT;
+        mbar_wait(&bars->kv_full[slot], (last / C::NSLOT) & 1, 62);
+      }
+    } else if (warp == kMmaWarp && lane == 0) {
+      const uint64_t d0 = sdesc_sw128(smem_u32(smem), 16, 1024);
+      constexpr uint64_t kToMn = (uint64_t)((C::CHUNK >> 4) - 1) << 16;
+      // a GEMM with A = Q or dO from tensor memory and B = a K-major ring tile
+      auto issue_tn = [&](uint32_t d_tmem, uint32_t a_tmem, int slot) {
+        const uint64_t b = sdesc_at(opaque(d0), C::OFF_RING + slot * C::TILE);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+          mma_ts(d_tmem, a_tmem + kk * 8, sdesc_at(b, koff), C::IDESC_S, kk > 0);
+        }
+      };
+      bool ok = n > 0 && mbar_wait(&bars->q_ready, 0, 63);
+      auto wait_slot = [&](int s2) {
+        return mbar_wait(&bars->kv_full[s2 % C::NSLOT], (uint32_t)((s2 / C::NSLOT) & 1), 64);
+      };
+      if (ok) ok = wait_slot(0);
+      if (ok) {
+        tc_fence_after();
+        issue_tn(tmem + C::T_S, tmem + C::T_Q, 0);  // S_0
+        mma_commit(&bars->s_full);
+        ok = wait_slot(1);
+      }
+      if (ok) {
+        tc_fence_after();
+        issue_tn(tmem + C::T_DP, tmem + C::T_DO, 1 % C::NSLOT);  // dP_0
+        mma_commit(&bars->dp_full);
+        mma_commit(&bars->kv_empty[1 % C::NSLOT]);
+      }
+      for (int j = 0; j < n && ok; ++j) {
+        const int kslot = (2 * j) % C::NSLOT;
+        if (j + 1 < n) {
+          // S_{j+1} over S_j once the dS warps have read S_j
+          ok = mbar_wait(&bars->s_free, j & 1, 65);
+          if (ok) ok = wait_slot(2 * j + 2);
+          if (!ok) break;
+          tc_fence_after();
+          issue_tn(tmem + C::T_S, tmem + C::T_Q, (2 * j + 2) % C::NSLOT);
+          mma_commit(&bars->s_full);
+        }
+        ok = mbar_wait(&bars->ds_full, j & 1, 66);
+        if (!ok) break;
+        tc_fence_after();
+        // dQ += dS_j K_j : A = dS (tensor memory, keys 64h.. at dP + 64h), B = K_j MN-major
+        {
+          const uint64_t b = sdesc_at(opaque(d0), C::OFF_RING + kslot * C::TILE) + kToMn;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_ts(tmem + C::T_DQ, tmem + C::T_DP + 64 * (kk / 4) + 8 * (kk % 4), sdesc_at(b, kk * 2048),
+                   C::IDESC_DQ, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&bars->kv_empty[kslot]);
+        if (j + 1 < n) {
+          // dP_{j+1} over dP_j / dS_j: issued after dQ_j, which reads dS_j first
+          ok = wait_slot(2 * j + 3);
+          if (!ok) break;
+          tc_fence_after();
+          issue_tn(tmem + C::T_DP, tmem + C::T_DO, (2 * j + 3) % C::NSLOT);
+          mma_commit(&bars->dp_full);
+          mma_commit(&bars->kv_empty[(2 * j + 3) % C::NSLOT]);
+        }
+      }
+      mma_commit(&bars->dq_done);
+      mma_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, 67);
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsCompute));
+    const int qw = warp % 4, h = warp / 4;
+    const int r = qw * 32 + lane;  // query row in the tile
+    const int q_row = i * BM + r;
+    const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
+    bool ok = mbar_wait(&bars->q_full, 0, 68);
+    // Q and dO into tensor memory: this warp copies half of its 32 rows' bytes
+    // (the half-h columns) from the 128-byte swizzled TMA tiles
+    if (ok) {
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t base = smem_u32(smem + (which ? C::OFF_DO : C::OFF_Q));
+        const uint32_t tdst = tmem + lane_off + (which ? C::T_DO : C::T_Q);
+        constexpr int UNITS = D / 16;  // 16-byte units of this warp's half row (D/2 bf16)
+        uint32_t v[UNITS * 4];
+#pragma unroll
+        for (int u = 0; u < UNITS; ++u) {
+          const int gu = h * UNITS + u;  // 16-byte unit of the whole row
+          const uint32_t chunk = gu / 8, within = gu % 8;
+          const float4 f = ld_shared_v4(base + chunk * C::CHUNK + r * 128 + ((within ^ (r & 7)) << 4));
+          v[4 * u] = __float_as_uint(f.x);
+          v[4 * u + 1] = __float_as_uint(f.y);
+          v[4 * u + 2] = __float_as_uint(f.z);
+          v[4 * u + 3] = __float_as_uint(f.w);
+        }
+        if constexpr (D == 128) {
+          tmem_st32(tdst + h * 32, v);
+        } else {
+          tmem_st16(tdst + h * 16, v);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->q_ready);
+    }
+    const float lse2 = sVec[r], dsm = sVec[BM + r];
+    const float c = p.scale_log2;
+    const uint32_t tS = tmem + lane_off + C::T_S + 64 * h;
+    const uint32_t tDP = tmem + lane_off + C::T_DP + 64 * h;
+    for (int j = 0; j < n && ok; ++j) {
+      ok = mbar_wait(&bars->s_full, j & 1, 69);
+      if (!ok) break;
+      tc_fence_after();
+      float pr[64];
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tS + cc * 32, v);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) pr[cc * 32 + e] = __uint_as_float(v[e]);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&bars->s_free);
+      // keys j*BN + 64h + col: hidden past Nk, or above the causal diagonal
+      const int k0 = j * BN + 64 * h;
+      const int lim = p.causal ? min(q_row + 1 + p.off, p.Nk) : p.Nk;  // keys < lim visible
+      if (k0 + 64 > lim) {
+#pragma unroll
+        for (int col = 0; col < 64; ++col)
+          if (k0 + col >= lim) pr[col] = -INFINITY;
+      }
+      const uint64_t c2 = f2_pack(c, c), l2 = f2_pack(lse2, lse2);
+#pragma unroll
+      for (int e = 0; e < 64; e += 2) {
+        float x0, x1;
+        f2_unpack(f2_fma(f2_pack(pr[e], pr[e + 1]), c2, l2), x0, x1);
+        pr[e] = ex2(x0);
+        pr[e + 1] = ex2(x1);
+      }
+      ok = mbar_wait(&bars->dp_full, j & 1, 70);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t w[32];
+      const uint64_t d2 = f2_pack(dsm, dsm);
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tDP + cc * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float a, b;
+          f2_unpack(f2_mul(f2_pack(pr[cc * 32 + e], pr[cc * 32 + e + 1]),
+                           f2_add(f2_pack(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), d2)),
+                    a, b);
+          w[cc * 16 + e / 2] = pack_bf16x2(a, b);
+        }
+      }
+      // dS (bf16, 64 keys) over the first 32 of this warp's own dP columns
+      tmem_st32(tDP, w);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars->ds_full);
+    }
+    if (ok) ok = n == 0 || mbar_wait(&bars->dq_done, 0, 71);
+    if (ok) {
+      tc_fence_after();
+      constexpr int DH = D / 2;  // dQ columns per warp
+      const bool row_ok = q_row < p.Nq;
+      __nv_bfloat16* dst = p.dq + ((size_t)bh * p.Nq + (row_ok ? q_row : 0)) * D + h * DH;
+      if (n == 0) {
+        if (row_ok) {
+#pragma unroll
+          for (int u = 0; u < DH / 8; ++u) reinterpret_cast<uint4*>(dst)[u] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      } else {
+        // every lane takes part in the tensor-memory loads (.sync.aligned);
+        // only rows inside the problem store
+#pragma unroll
+        for (int cc = 0; cc < DH / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tmem + lane_off + C::T_DQ + h * DH + cc * 32, v);
+          tmem_wait_ld();
+          if (row_ok) {
+            uint32_t o[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              o[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * p.scale, __uint_as_float(v[2 * e + 1]) * p.scale);
+            uint4* o4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) o4[u] = make_uint4(o[4 * u], o[4 * u + 1], o[4 * u + 2], o[4 * u + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Query heads per locality chunk of the dQ pass: per query head the pass reads
+// its Q and dO once and the K and V of its key/value head for every query tile
+// (4 Nk d bytes per key/value head); a chunk keeps its K and V near 40 MB of L2
+// and holds at least two waves of CTAs.
+inline int chunk_heads(int BH, int G, int Nk, int d, int nq, int sms) {
+  const long long kv_head = 4LL * Nk * d;
+  long long c = std::max(1LL, (40LL << 20) / kv_head) * G;
+  c = std::max<long long>(c, (2LL * sms + nq - 1) / nq);
+  c = std::min<long long>(((c + G - 1) / G) * G, BH);
+  const long long nch = (BH + c - 1) / c;
+  c = (BH + nch - 1) / nch;
+  return (int)std::min<long long>(((c + G - 1) / G) * G, BH);
+}
+
+}  // namespace dqp
 
 // Key/value heads per locality chunk.  Per key/value head the pass touches
 // K and V (4 Nk d bytes), the Q and dO of its G query heads (4 G Nq d bytes) and
@@ -661,6 +1058,33 @@ size_t sm100_backward_dq_offset(int BH, int N) {
   return 2 * (((size_t)BH * npad * 4 + 255) / 256 * 256);
 }
 
+namespace {
+
+template <int D, bool kDQ>
+cudaError_t launch_main(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        const CUtensorMap& mdo, const CUtensorMap& mdq, const bwd::Params& p,
+                        cudaStream_t st) {
+  const int smem = bwd::Cfg<D>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(bwd::main_kernel<D, kDQ>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  bwd::main_kernel<D, kDQ><<<grid, bwd::NTHREADS, smem, st>>>(mq, mk, mv, mdo, mdq, p);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_dq(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      const CUtensorMap& mdo, const bwd::dqp::Params& p, cudaStream_t st) {
+  const int smem = bwd::dqp::Cfg<D>::SMEM_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(bwd::dqp::dq_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  bwd::dqp::dq_kernel<D><<<grid, bwd::dqp::NTHREADS, smem, st>>>(mq, mk, mv, mdo, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                            const CUtensorMap& mdo, const CUtensorMap& mdq, const void* o,
                            const void* dout, const float* lse,
@@ -669,68 +1093,92 @@ cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const C
                            cudaStream_t st) {
   const int BH = B * H;
   const int N = Nq;  // the workspace and the preprocess run over query rows
+  const bool det = (stages & kStageDeterministic) != 0;
   const int npad = (N + 127) / 128 * 128;
   const size_t vec = ((size_t)BH * npad * 4 + 255) / 256 * 256;
   float* lse2 = static_cast<float*>(workspace);
   float* dsum = reinterpret_cast<float*>(static_cast<char*>(workspace) + vec);
   float* acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * vec);
   cudaError_t e = cudaSuccess;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  sms = std::max(sms, 1);
   if (stages & kStagePreprocess) {
     const long long rows = (long long)BH * npad;
     const long long rows_per_block = 8LL * (256 / d);  // 8 warps of 256/d rows
     const unsigned pblocks = (unsigned)((rows + rows_per_block - 1) / rows_per_block);
-    if (d == 128)
-      bwd::preprocess_kernel<128><<<pblocks, 256, 0, st>>>(
-          (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, lse2, dsum, acc, BH, N, npad);
-    else
-      bwd::preprocess_kernel<64><<<pblocks, 256, 0, st>>>(
-          (const __nv_bfloat16*)o, (const __nv_bfloat16*)dout, lse, lse2, dsum, acc, BH, N, npad);
+    const auto* ob = static_cast<const __nv_bfloat16*>(o);
+    const auto* gb = static_cast<const __nv_bfloat16*>(dout);
+    if (d == 128) {
+      if (det)
+        bwd::preprocess_kernel<128, false><<<pblocks, 256, 0, st>>>(ob, gb, lse, lse2, dsum, acc, BH, N, npad);
+      else
+        bwd::preprocess_kernel<128, true><<<pblocks, 256, 0, st>>>(ob, gb, lse, lse2, dsum, acc, BH, N, npad);
+    } else {
+      if (det)
+        bwd::preprocess_kernel<64, false><<<pblocks, 256, 0, st>>>(ob, gb, lse, lse2, dsum, acc, BH, N, npad);
+      else
+        bwd::preprocess_kernel<64, true><<<pblocks, 256, 0, st>>>(ob, gb, lse, lse2, dsum, acc, BH, N, npad);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (!(stages & (kStageMain | kStageConvert))) return cudaSuccess;
-
-  bwd::Params p;
-  p.dk = static_cast<__nv_bfloat16*>(dk);
-  p.dv = static_cast<__nv_bfloat16*>(dv);
-  p.dq_acc = acc;
-  p.lse2 = lse2;
-  p.dsum = dsum;
-  p.BH = BH;
-  p.BHkv = B * Hkv;
-  p.H = H;
-  p.G = H / Hkv;
-  p.Nq = Nq;
-  p.Nk = Nk;
-  p.off = Nk - Nq;
-  p.Npad = npad;
-  p.nq = npad / 128;
-  p.nkv = (Nk + 127) / 128;
-  p.scale = scale;
-  p.scale_log2 = scale * bwd::kLog2e;
-  p.causal = causal;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  p.chunk = bwd::chunk_heads(p.BHkv, p.G, Nq, Nk, d, p.nkv, std::max(sms, 1));
-  const dim3 grid((unsigned)(p.nkv * p.BHkv));
-  if (!(stages & kStageMain)) {
-  } else if (d == 128) {
-    const int smem = bwd::Cfg<128>::SMEM_BYTES;
-    e = cudaFuncSetAttribute(bwd::main_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (stages & kStageMain) {
+    bwd::Params p;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.dq_acc = acc;
+    p.lse2 = lse2;
+    p.dsum = dsum;
+    p.BH = BH;
+    p.BHkv = B * Hkv;
+    p.H = H;
+    p.G = H / Hkv;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.off = Nk - Nq;
+    p.Npad = npad;
+    p.nq = npad / 128;
+    p.nkv = (Nk + 127) / 128;
+    p.scale = scale;
+    p.scale_log2 = scale * bwd::kLog2e;
+    p.causal = causal;
+    p.chunk = bwd::chunk_heads(p.BHkv, p.G, Nq, Nk, d, p.nkv, sms);
+    const dim3 grid((unsigned)(p.nkv * p.BHkv));
+    if (det)
+      e = d == 128 ? launch_main<128, false>(grid, mq, mk, mv, mdo, mdq, p, st)
+                   : launch_main<64, false>(grid, mq, mk, mv, mdo, mdq, p, st);
+    else
+      e = d == 128 ? launch_main<128, true>(grid, mq, mk, mv, mdo, mdq, p, st)
+                   : launch_main<64, true>(grid, mq, mk, mv, mdo, mdq, p, st);
     if (e != cudaSuccess) return e;
-    bwd::main_kernel<128><<<grid, bwd::NTHREADS, smem, st>>>(mq, mk, mv, mdo, mdq, p);
-  } else {
-    const int smem = bwd::Cfg<64>::SMEM_BYTES;
-    e = cudaFuncSetAttribute(bwd::main_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    bwd::main_kernel<64><<<grid, bwd::NTHREADS, smem, st>>>(mq, mk, mv, mdo, mdq, p);
   }
-  e = cudaGetLastError();
-  if (e != cudaSuccess || !(stages & kStageConvert)) return e;
-  const long long n8 = (long long)BH * N * d / 8;
-  const unsigned cblocks = (unsigned)std::min<long long>((n8 + 255) / 256, (long long)std::max(sms, 1) * 8);
-  bwd::dq_convert_kernel<<<cblocks, 256, 0, st>>>(acc, static_cast<__nv_bfloat16*>(dq), n8, scale);
+  if (!(stages & kStageConvert)) return cudaSuccess;
+  if (det) {
+    bwd::dqp::Params p;
+    p.dq = static_cast<__nv_bfloat16*>(dq);
+    p.lse2 = lse2;
+    p.dsum = dsum;
+    p.BH = BH;
+    p.H = H;
+    p.G = H / Hkv;
+    p.Nq = Nq;
+    p.Nk = Nk;
+    p.off = Nk - Nq;
+    p.Npad = npad;
+    p.nq = npad / 128;
+    p.causal = causal;
+    p.scale = scale;
+    p.scale_log2 = scale * bwd::kLog2e;
+    p.chunk = bwd::dqp::chunk_heads(BH, p.G, Nk, d, p.nq, sms);
+    const dim3 grid((unsigned)(p.nq * BH));
+    return d == 128 ? launch_dq<128>(grid, mq, mk, mv, mdo, p, st)
+                    : launch_dq<64>(grid, mq, mk, mv, mdo, p, st);
+  }
+  const long long n16 = (long long)BH * N * d / 16;
+  const unsigned cblocks = (unsigned)std::min<long long>((n16 + 255) / 256, (long long)sms * 16);
+  bwd::dq_convert_kernel<<<cblocks, 256, 0, st>>>(acc, static_cast<__nv_bfloat16*>(dq), n16, scale);
   return cudaGetLastError();
 }
 

@@ -46,7 +46,10 @@ size_t sm100_backward_dq_offset(int BH, int N);
 // `stages` selects the launches (kStagePreprocess | kStageMain | kStageConvert
 // for the whole pass); each later stage reads what the earlier ones left in the
 // workspace.
+// With kStageDeterministic the preprocess leaves the accumulator alone, the main
+// stage computes dK and dV only, and the last stage is the separate dQ pass.
 constexpr int kStagePreprocess = 1, kStageMain = 2, kStageConvert = 4, kStageAll = 7;
+constexpr int kStageDeterministic = 8;
 // mq, mdo, mdq over Nq rows; mk, mv over Nk rows.
 // mdq: 3-D fp32 view {d, Nq, B*H} of the accumulator, box {32, 32, 1}, 128-byte swizzle
 cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,

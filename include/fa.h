@@ -151,6 +151,20 @@ fa_status fa_backward_qk(const void* q, const void* k, const void* v, const void
                          void* workspace, size_t ws_bytes, int B, int H, int Hkv, int Nq, int Nk,
                          int d, float scale, int causal, void* stream);
 
+/* Deterministic backward pass: results as fa_backward_qk (Hkv = H and Nq = Nk
+ * give fa_backward), computed so that they are the same bit for bit from run to
+ * run.  dK and dV come from one CTA per key tile as always; dQ comes from a
+ * separate pass, one CTA per 128-row query tile that walks its key tiles in a
+ * fixed order and sums dS K in tensor memory, instead of partial sums added
+ * into an fp32 accumulator in whatever order the CTAs finish.  It executes
+ * 7 N^2 d multiply-adds per head instead of 5 (S and dP are formed twice), and
+ * the workspace (same size rule as fa_backward) holds only the LSE and D rows.
+ * Errors as fa_backward. */
+fa_status fa_backward_deterministic(const void* q, const void* k, const void* v, const void* o,
+                                   const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                   void* workspace, size_t ws_bytes, int B, int H, int Hkv, int Nq,
+                                   int Nk, int d, float scale, int causal, void* stream);
+
 /* Stages of the bf16 backward pass, for callers that schedule or time them one
  * by one (fa_backward runs all three in one call):
  *   FA_STAGE_PREPROCESS  -LSE*log2(e) and -D_i = -sum_c dO[i,c] O[i,c] into the
@@ -159,14 +173,19 @@ fa_status fa_backward_qk(const void* q, const void* k, const void* v, const void
  *                        partial dQ = dS K of every key tile added into the
  *                        accumulator;
  *   FA_STAGE_DQ_CONVERT  dQ = scale * accumulator, rounded to bf16.
+ * With FA_STAGE_DETERMINISTIC added, the stages are those of
+ * fa_backward_deterministic: the preprocess leaves no accumulator, the main
+ * stage writes dK and dV only, and FA_STAGE_DQ_CONVERT runs the separate dQ pass.
  * Arguments as fa_backward_qk (Hkv = H and Nq = Nk for the square multi-head
- * case) plus `stages`, a nonzero OR of the flags.  A later stage reads what an
+ * case) plus `stages`, a nonzero OR of the three stage flags, optionally with
+ * FA_STAGE_DETERMINISTIC (the same choice for every stage of one backward).  A later stage reads what an
  * earlier one left in the workspace, so run them in this order, on one stream
  * (or ordered by events), with the same arguments and workspace and nothing
  * else writing the workspace in between. */
 #define FA_STAGE_PREPROCESS 1
 #define FA_STAGE_MAIN 2
 #define FA_STAGE_DQ_CONVERT 4
+#define FA_STAGE_DETERMINISTIC 8
 fa_status fa_backward_stages(const void* q, const void* k, const void* v, const void* o,
                              const void* dout, const float* lse, void* dq, void* dk, void* dv,
                              void* workspace, size_t ws_bytes, int B, int H, int Hkv, int Nq,

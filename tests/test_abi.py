@@ -136,7 +136,7 @@ def test_backward_stages_rejects_bad_arguments(lib):
     ptrs = [P(0x10000 * (i + 1)) for i in range(9)]
     ws = P(0x100000)
     need = lib.fa_backward_workspace_size(1, 4, 100, 64)
-    for stages in (0, 8, -1, 15):
+    for stages in (0, 8, -1, 16, 24, 0x107):
         assert f(*ptrs, ws, need, 1, 4, 2, 100, 300, 64, 0.125, 1, stages, None) == INVALID
     assert f(*ptrs, ws, need - 1, 1, 4, 2, 100, 300, 64, 0.125, 1, 2, None) == WORKSPACE
     assert f(*ptrs, P(0x100004), need, 1, 4, 2, 100, 300, 64, 0.125, 1, 2, None) == MISALIGNED
@@ -205,3 +205,18 @@ def test_fp8_forward_rejects_bad_arguments(lib):
     ptrs = list(GOOD)
     ptrs[1] = P(0x20001)
     assert f(*ptrs, 1, 2, 1, 16, 16, 64, 0.125, *good, 0, None) == MISALIGNED
+
+
+def test_deterministic_backward_rejects_bad_arguments(lib):
+    f = lib.fa_backward_deterministic
+    ptrs = [P(0x10000 * (i + 1)) for i in range(9)]
+    ws = P(0x100000)
+    need = lib.fa_backward_workspace_size(1, 4, 100, 64)
+    assert f(*ptrs, ws, need - 1, 1, 4, 2, 100, 300, 64, 0.125, 1, None) == WORKSPACE
+    assert f(*ptrs, P(0x100004), need, 1, 4, 2, 100, 300, 64, 0.125, 1, None) == MISALIGNED
+    assert f(*ptrs, ws, need, 1, 4, 3, 100, 300, 64, 0.125, 1, None) == INVALID
+    assert f(*ptrs, ws, need, 1, 4, 2, 100, 300, 96, 0.125, 1, None) == UNSUPPORTED
+    for i in range(9):
+        bad = list(ptrs)
+        bad[i] = None
+        assert f(*bad, ws, need, 1, 4, 2, 100, 300, 64, 0.125, 1, None) == INVALID
