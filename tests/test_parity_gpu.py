@@ -281,3 +281,22 @@ def test_fewer_queries_are_the_last_rows_of_the_square_case_on_gpu():
     o, lse = fa.forward_qk(qd[:, :, 1000 - 300 :].contiguous(), kd, vd, causal=True)
     assert max_abs(to_f64(o), to_f64(o_sq[:, :, 700:])) <= 1e-2
     assert max_abs(to_f64(lse), to_f64(l_sq[:, :, 700:])) <= 1e-4
+
+
+def test_forward_permutation_equivariance_on_gpu():
+    # non-causal attention commutes with permutations: permuting the queries
+    # permutes the output rows (bit for bit: every row is computed on its own),
+    # and permuting keys together with values leaves O and LSE unchanged up to
+    # the summation order
+    B, H, N, d = 1, 3, 700, 128
+    q, k, v = (t.cuda() for t in make_inputs(B, H, N, d, seed=31))
+    g = torch.Generator().manual_seed(5)
+    perm_q = torch.randperm(N, generator=g).cuda()
+    perm_k = torch.randperm(N, generator=g).cuda()
+    o, lse = fa.forward(q, k, v)
+    oq, lq = fa.forward(q[:, :, perm_q].contiguous(), k, v)
+    assert torch.equal(oq, o[:, :, perm_q]) and torch.equal(lq, lse[:, :, perm_q])
+    ok_, lk = fa.forward(q, k[:, :, perm_k].contiguous(), v[:, :, perm_k].contiguous())
+    fa.check_device_status()
+    assert max_abs(to_f64(ok_), to_f64(o)) <= O_MAXABS
+    assert max_abs(to_f64(lk), to_f64(lse)) <= 1e-4
