@@ -300,3 +300,65 @@ def test_forward_permutation_equivariance_on_gpu():
     fa.check_device_status()
     assert max_abs(to_f64(ok_), to_f64(o)) <= O_MAXABS
     assert max_abs(to_f64(lk), to_f64(lse)) <= 1e-4
+
+
+# ---------------------------------------------------------------- sizes at the edges
+
+
+def test_many_heads_small_tiles():
+    # 8192 heads of one 128-row tile: thousands of work items through the
+    # forward's scheduler and 8192 backward CTAs, checked on a spread of heads
+    B, H, N, d = 2, 4096, 128, 64
+    q, k, v, do = (t.cuda() for t in make_inputs(B, H, N, d, seed=41, with_do=True))
+    o = torch.full_like(q, float("nan"))
+    lse = torch.full((B, H, N), float("nan"), device="cuda")
+    fa.forward(q, k, v, causal=True, out=o, lse=lse)
+    dq, dk, dv = (torch.full_like(t, float("nan")) for t in (q, k, v))
+    fa.backward(q, k, v, o, do, lse, causal=True, dq=dq, dk=dk, dv=dv)
+    fa.check_device_status()
+    for t in (o, lse, dq, dk, dv):
+        assert not bool(torch.isnan(t).any())
+    for b, h in [(0, 0), (0, 4095), (1, 1234), (1, 4095)]:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        args = [to_f64(x[sl].cpu()) for x in (q, k, v)]
+        o_ref, lse_ref = attention_fwd_ref(*args, 1 / math.sqrt(d), True)
+        check_fwd(to_f64(o[sl]), to_f64(lse[sl]), o_ref, lse_ref, (b, h))
+        ref = attention_bwd_ref(*args, to_f64(do[sl].cpu()), 1 / math.sqrt(d), True)
+        check_bwd([to_f64(g[sl]) for g in (dq, dk, dv)], ref, (b, h))
+
+
+def test_long_single_head_forward_sampled_rows():
+    # one head of 131072 keys (causal): 512 query-tile pairs in one head
+    from exact_tiled_attention_35_b200.inputs import sample_rows
+    from oracle import attention_rows_ref
+
+    B, H, N, d = 1, 1, 131072, 128
+    q, k, v = make_inputs(B, H, N, d, seed=43)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    o = torch.full_like(qd, float("nan"))
+    lse = torch.full((B, H, N), float("nan"), device="cuda")
+    fa.forward(qd, kd, vd, causal=True, out=o, lse=lse)
+    fa.check_device_status()
+    assert not bool(torch.isnan(o).any()) and not bool(torch.isnan(lse).any())
+    rows = [sample_rows(N, 48, 43, 0)]
+    o_ref, lse_ref = attention_rows_ref(to_f64(q), to_f64(k), to_f64(v), rows, 1 / math.sqrt(d), True)
+    check_fwd(to_f64(o)[:, :, rows[0]], to_f64(lse)[:, :, rows[0]], o_ref, lse_ref, "N=131072")
+
+
+@pytest.mark.parametrize("N", [129, 255, 257, 383])
+def test_one_row_past_a_tile_boundary(N):
+    # ragged tails one row either side of a tile edge, grouped heads, both passes
+    from oracle import attention_bwd_gqa_ref, attention_fwd_gqa_ref
+
+    q, do = make_inputs(1, 4, N, 128, seed=N, with_do=True)[0::3]
+    k, v = make_inputs(1, 2, N, 128, seed=N + 1)[1:3]
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    o, lse = fa.forward_gqa(qd, kd, vd, causal=True)
+    dq, dk, dv = (torch.full_like(t, float("nan")) for t in (qd, kd, vd))
+    fa.backward_gqa(qd, kd, vd, o, dod, lse, causal=True, dq=dq, dk=dk, dv=dv)
+    fa.check_device_status()
+    args = (to_f64(q), to_f64(k), to_f64(v))
+    o_ref, lse_ref = attention_fwd_gqa_ref(*args, 1 / math.sqrt(128), True)
+    check_fwd(to_f64(o), to_f64(lse), o_ref, lse_ref, N)
+    ref = attention_bwd_gqa_ref(*args, to_f64(do), 1 / math.sqrt(128), True)
+    check_bwd([to_f64(x) for x in (dq, dk, dv)], ref, N)
