@@ -67,14 +67,14 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return g_encode;
 }
 
-// 3-D bf16 view {d, N, B*H} of a [B,H,N,d] tensor, box {64, 128, 1}, 128-byte
-// swizzle; rows past N read as zero.
-bool make_map(CUtensorMap* map, const void* base, int d, int N, int BH) {
+// 3-D bf16 view {d, N, B*H} of a [B,H,N,d] tensor, box {64, rows, 1}, 128-byte
+// swizzle; rows past N read as zero (loads) or are not written (stores).
+bool make_map(CUtensorMap* map, const void* base, int d, int N, int BH, unsigned rows = 128) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = encoder();
   if (!enc) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
   const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -191,12 +191,13 @@ fa_status backward_bf16(const void* q, const void* k, const void* v, const void*
                         void* workspace, int B, int H, int Hkv, int Nq, int Nk, int d,
                         float scale, int causal, int stages, void* stream) {
   const int BH = B * H;
-  CUtensorMap mq, mk, mv, mdo, mdq;
+  CUtensorMap mq, mk, mv, mdo, mdq, mdk, mdv;
   if (!make_map(&mq, q, d, Nq, BH) || !make_map(&mk, k, d, Nk, B * Hkv) ||
       !make_map(&mv, v, d, Nk, B * Hkv) || !make_map(&mdo, dout, d, Nq, BH) ||
-      !make_dq_map(&mdq, static_cast<char*>(workspace) + sm100_backward_dq_offset(BH, Nq), d, Nq, BH))
+      !make_dq_map(&mdq, static_cast<char*>(workspace) + sm100_backward_dq_offset(BH, Nq), d, Nq, BH) ||
+      !make_map(&mdk, dk, d, Nk, B * Hkv, 32) || !make_map(&mdv, dv, d, Nk, B * Hkv, 32))
     return map_failed();
-  return from_cuda(sm100_backward(mq, mk, mv, mdo, mdq, o, dout, lse, dq, dk, dv, workspace, B, H,
+  return from_cuda(sm100_backward(mq, mk, mv, mdo, mdq, mdk, mdv, o, dout, lse, dq, dk, dv, workspace, B, H,
                                   Hkv, Nq, Nk, d, scale, causal ? 1 : 0, stages,
                                   static_cast<cudaStream_t>(stream)));
 }

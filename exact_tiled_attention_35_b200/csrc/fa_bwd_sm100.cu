@@ -8,23 +8,26 @@
 //
 // Three kernels:
 //   preprocess  -D and -LSE * log2(e) (padded to whole 128-row tiles: padding
-//               rows get +inf for LSE so their probabilities vanish) and a zeroed
-//               fp32 dQ accumulator;
-//   main        one CTA per 128-key tile; for every 128-row query tile it
-//               recomputes S^T = K Q^T and dP^T = V dO^T in tensor memory,
-//               forms P^T (to tensor memory) and dS (to shared memory), then
-//               accumulates dV += P^T dO and dK += dS^T Q in tensor memory and
-//               computes the partial dQ = dS K, which a reduce group adds into
-//               the fp32 accumulator with bulk tensor reduce-adds;
+//               rows get +inf for LSE so their probabilities vanish), a zeroed
+//               fp32 dQ accumulator and the main kernel's zeroed ticket counters;
+//   main        persistent, one CTA per SM; a work item is one 128-key tile of
+//               one key/value head.  For every 128-row query tile it recomputes
+//               S^T = K Q^T and dP^T = V dO^T in tensor memory, forms P^T (to
+//               tensor memory) and dS (to shared memory), then accumulates
+//               dV += P^T dO and dK += dS^T Q in tensor memory and computes the
+//               partial dQ = dS K, which a reduce group adds into the fp32
+//               accumulator with bulk tensor reduce-adds;
 //   convert     dQ = scale * accumulator, rounded to bf16.
 //
 // Main-kernel CTA layout (512 threads, registers rebalanced with setmaxnreg):
 //   warps 0-7   P / dS computation (thread = key row = tensor-memory lane, two
 //               warps per row quarter, one per half of the query columns) and
-//               the dK / dV epilogue
+//               the dK / dV epilogue (TMA stores of 32-row boxes)
 //   warps 8-11  dQ drain: tensor memory -> registers -> shared staging -> bulk
 //               tensor reduce-add into the fp32 accumulator
-//   warp  12    TMA producer: K, V once; Q_i, dO_i, LSE_i, D_i per query tile
+//   warp  12    TMA producer: draws work items; K, V once per item (prefetched
+//               into L2 when the item is drawn); Q_i, dO_i, LSE_i, D_i per
+//               query tile
 //   warp  13    tensor-memory allocator and MMA issuer (warps 14-15 idle)
 // Tensor memory: S^T at column 0 (P^T of query columns 64h.. packed at column 64h),
 // dP^T / dQ at 128, dV at 256, dK at 256+d.
@@ -97,13 +100,18 @@ struct Params {
   int nq;              // number of query tiles = Npad / 128
   int nkv;             // number of key tiles
   int chunk;           // key/value heads per locality chunk
+  int items;           // work items: key tiles x key/value heads
+  unsigned long long* tickets;  // [0] items handed out past the first gridDim.x, [1] CTAs done
   float scale;
   float scale_log2;
   int causal;
 };
 
+constexpr int kItemRing = 2;  // work items the producer may hand out ahead
+
 struct Bars {
   uint64_t kv_full;
+  uint64_t kv_empty;       // the item's last GEMM reading K or V has completed
   uint64_t q_full[NST];    // Q tile + LSE2 / D vectors of a stage
   uint64_t q_empty[NST];
   uint64_t do_full;        // dO tile (single buffer)
@@ -115,10 +123,43 @@ struct Bars {
   uint64_t ds_free;
   uint64_t dq_full;
   uint64_t dq_empty;
-  uint64_t all_done;
+  uint64_t acc_full;       // the item's dK and dV are complete in tensor memory
   uint64_t drain;
+  uint64_t it_full[kItemRing];   // the producer has written it_item[s]
+  uint64_t it_empty[kItemRing];  // every reader has taken it_item[s]
+  int it_item[kItemRing];
   uint32_t tmem_base;
 };
+static_assert(sizeof(Bars) <= 256, "barrier block over its shared-memory slot");
+
+// Work item -> key tile j and key/value head.  The key/value heads are cut into
+// chunks whose K, V, Q, dO and fp32 dQ accumulator fit in L2 together; chunk by
+// chunk, items run key-tile-major, so under the causal mask (tile j sees query
+// tiles from about j on) the heavy items come first, and CTAs take them in
+// this order as they become free.
+struct Item {
+  int j;      // key tile
+  int bkv;    // key/value head
+  int i0;     // first query tile with a row that sees a key of tile j
+  int nqi;    // query tiles per query head
+  int niter;  // query tiles of the item: every query head of the group
+  int bhq0;   // first query head of the group
+};
+
+__device__ __forceinline__ Item decode_item(const Params& p, int item) {
+  const int per_chunk = p.chunk * p.nkv;
+  const int chunk_id = item / per_chunk, w_in = item - chunk_id * per_chunk;
+  const int h0 = chunk_id * p.chunk, hn = min(p.chunk, p.BHkv - h0);
+  Item w;
+  w.j = w_in / hn;
+  w.bkv = h0 + (w_in - w.j * hn);
+  // the causal mask is aligned bottom right: key k is visible to query r iff k <= r + off
+  w.i0 = p.causal ? max(0, w.j * BN - p.off) / BM : 0;
+  w.nqi = p.nq - w.i0;
+  w.niter = p.G * w.nqi;
+  w.bhq0 = (w.bkv / (p.H / p.G)) * p.H + (w.bkv % (p.H / p.G)) * p.G;
+  return w;
+}
 
 
 // Bulk tensor reduce-add of a shared-memory box into global memory (async proxy).
@@ -137,6 +178,22 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
           smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Bulk tensor store of a shared-memory box (async proxy; completion by bulk group).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src_smem, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src_smem), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
+// Fetch a box into L2 only (no shared memory, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
 }
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -160,11 +217,19 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // kDQ: also form the partial dQ = dS K of every query tile and add it into the
 // fp32 accumulator (the single-pass backward); without it the kernel computes
 // dK and dV only and dQ comes from dq_kernel.
+//
+// Persistent: one CTA per SM takes work items (key/value head, 128-key tile) in
+// the order of decode_item, its first item b = blockIdx.x and every later one
+// from the launch's ticket counter.  Barrier phases, the Q / dO stages and the
+// tensor-memory buffers carry over from item to item, so the next item's loads
+// and first GEMMs overlap the current item's last dQ reduction and its dK / dV
+// epilogue.
 template <int D, bool kDQ>
 __global__ void __launch_bounds__(NTHREADS, 1)
     main_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                 const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mdo,
-                const __grid_constant__ CUtensorMap mdq, const Params p) {
+                const __grid_constant__ CUtensorMap mdq, const __grid_constant__ CUtensorMap mdk,
+                const __grid_constant__ CUtensorMap mdv, const Params p) {
   using C = Cfg<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
   // The swizzled tiles need a 1024-byte aligned base and the layout uses the
@@ -181,30 +246,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  // CTA -> (key/value head, key tile).  The heads are cut into chunks whose
-  // K, V, Q, dO and fp32 dQ accumulator fit in L2 together; chunk by chunk,
-  // CTAs run key-tile-major with the heavy tiles first under the causal mask
-  // (tile j sees query tiles j..), and the block scheduler hands them to SMs in
-  // that order as SMs free up.
-  const int blk = blockIdx.x;
-  const int per_chunk = p.chunk * p.nkv;
-  const int chunk_id = blk / per_chunk, w_in = blk - chunk_id * per_chunk;
-  const int h0 = chunk_id * p.chunk, hn = min(p.chunk, p.BHkv - h0);
-  const int j = w_in / hn;
-  const int bkv = h0 + (w_in - j * hn);  // key/value head
-  const int nq = p.nq;
-  // first query tile with a row that sees a key of tile j (the causal mask is
-  // aligned bottom right: key k visible to query r iff k <= r + off)
-  const int i0 = p.causal ? max(0, j * BN - p.off) / BM : 0;
-  const int nqi = nq - i0;        // query tiles per query head
-  const int niter = p.G * nqi;    // every query head of the group, then its query tiles
-  // query head and query tile of iteration it
-  const int bhq0 = (bkv / (p.H / p.G)) * p.H + (bkv % (p.H / p.G)) * p.G;
-  auto q_head = [&](int it) { return bhq0 + it / nqi; };
-  auto q_tile = [&](int it) { return i0 + it % nqi; };
+  constexpr int kItemReaders = kDQ ? 13 : 9;  // MMA warp, 8 compute warps (+ 4 reduce warps)
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
+    mbar_init(&bars->kv_empty, 1);
     for (int s = 0; s < NST; ++s) {
       mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->q_empty[s], 1);
@@ -218,8 +264,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     mbar_init(&bars->ds_free, 1);
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->dq_empty, 128);
-    mbar_init(&bars->all_done, 1);
+    mbar_init(&bars->acc_full, 1);
     mbar_init(&bars->drain, 1);
+    for (int s = 0; s < kItemRing; ++s) {
+      mbar_init(&bars->it_full[s], 1);
+      mbar_init(&bars->it_empty[s], kItemReaders);
+    }
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -232,28 +282,38 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tma_prefetch_desc(&mv);
     tma_prefetch_desc(&mdo);
     tma_prefetch_desc(&mdq);
+    tma_prefetch_desc(&mdk);
+    tma_prefetch_desc(&mdv);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
+  // The r-th work item of this CTA from the producer's ring (>= p.items: none
+  // left).  Every lane of the calling warp reads it; lane 0 then frees the entry.
+  auto take_item = [&](int r, int& item, unsigned int site) -> bool {
+    const int s = r % kItemRing;
+    if (!mbar_wait(&bars->it_full[s], (uint32_t)((r / kItemRing) & 1), site)) return false;
+    item = *reinterpret_cast<volatile int*>(&bars->it_item[s]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars->it_empty[s]);
+    return true;
+  };
+
   if (warp >= 12) {
    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsControl));
    if (warp == kProducerWarp) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(sK + c * C::CHUNK, &mk, &bars->kv_full, c * 64, j * BN, bkv);
-        tma_load_3d(sV + c * C::CHUNK, &mv, &bars->kv_full, c * 64, j * BN, bkv);
-      }
       bool ok = true;
-      int issued = 0, do_issued = 0;
-      for (int it = 0; it < niter && ok; ++it) {
-        const int st = it % NST, round = it / NST;
-        const int i = q_tile(it), bh = q_head(it);
-        if (round > 0) ok = mbar_wait(&bars->q_empty[st], (round - 1) & 1, 32);
-        if (!ok) break;
+      int g = 0;      // query tiles (Q, dO) loaded so far, over all items
+      int nkv = 0;    // items whose K and V were loaded
+      int dog = 0;    // dO tiles loaded
+      // loads of one query tile: Q, the LSE2 / D rows into stage g % NST, dO
+      auto load_tile = [&](const Item& w, int it) -> bool {
+        const int st = g % NST, round = g / NST;
+        const int i = w.i0 + it % w.nqi, bh = w.bhq0 + it / w.nqi;
+        if (round > 0 && !mbar_wait(&bars->q_empty[st], (round - 1) & 1, 32)) return false;
         uint8_t* sQ = smem + C::OFF_Q + st * C::TILE;
         float* vec = sVec + st * 2 * BM;
         mbar_arrive_expect_tx(&bars->q_full[st], C::TILE + 2 * BM * 4);
@@ -262,258 +322,354 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const size_t voff = (size_t)bh * p.Npad + (size_t)i * BM;
         bulk_load(vec, p.lse2 + voff, BM * 4, &bars->q_full[st]);
         bulk_load(vec + BM, p.dsum + voff, BM * 4, &bars->q_full[st]);
-        issued = it + 1;
-        // dO of tile i reuses the single dO buffer once dV of tile i-1 has read it
-        if (it > 0) ok = mbar_wait(&bars->do_empty, (it - 1) & 1, 47);
-        if (!ok) break;
+        ++g;
+        // dO of a tile reuses the single dO buffer once dV of the tile before has read it
+        if (dog > 0 && !mbar_wait(&bars->do_empty, (dog - 1) & 1, 47)) return false;
         mbar_arrive_expect_tx(&bars->do_full, C::TILE);
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d(smem + C::OFF_DO + c * C::CHUNK, &mdo, &bars->do_full, c * 64, i * BM, bh);
-        do_issued = it + 1;
+        ++dog;
+        return true;
+      };
+      for (int r = 0; ok; ++r) {
+        // A CTA draws its next item once it has issued the loads of the current
+        // one, about two query tiles before that item ends.
+        const int item = r == 0 ? (int)blockIdx.x : (int)gridDim.x + (int)atomicAdd(p.tickets, 1ull);
+        const int s = r % kItemRing;
+        if (r >= kItemRing) ok = mbar_wait(&bars->it_empty[s], (uint32_t)((r / kItemRing - 1) & 1), 50);
+        if (!ok) break;
+        *reinterpret_cast<volatile int*>(&bars->it_item[s]) = item;
+        mbar_arrive(&bars->it_full[s]);
+        if (item >= p.items) break;
+        const Item w = decode_item(p, item);
+        // K and V come from DRAM (each key tile is read by one item only); start
+        // bringing them into L2 now, while the current item still runs
+        if (r > 0)
+          for (int c = 0; c < D / 64; ++c) {
+            tma_prefetch_l2_3d(&mk, c * 64, w.j * BN, w.bkv);
+            tma_prefetch_l2_3d(&mv, c * 64, w.j * BN, w.bkv);
+          }
+        // the first query tile's Q and dO are fetched before K and V, whose
+        // buffers free only when the previous item's last GEMM reading them ends
+        ok = load_tile(w, 0);
+        if (ok && r > 0) ok = mbar_wait(&bars->kv_empty, (r - 1) & 1, 51);
+        if (!ok) break;
+        mbar_arrive_expect_tx(&bars->kv_full, 2 * C::TILE);
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(sK + c * C::CHUNK, &mk, &bars->kv_full, c * 64, w.j * BN, w.bkv);
+          tma_load_3d(sV + c * C::CHUNK, &mv, &bars->kv_full, c * 64, w.j * BN, w.bkv);
+        }
+        ++nkv;
+        for (int it = 1; it < w.niter && ok; ++it) ok = load_tile(w, it);
       }
-      mbar_wait(&bars->kv_full, 0, 33);
-      for (int s = 0; s < NST && s < issued; ++s) {
-        const int last = s + ((issued - 1 - s) / NST) * NST;
+      // This CTA draws no more tickets; the last one to get here resets the
+      // counters for the next launch on this workspace.
+      __threadfence();
+      if (atomicAdd(p.tickets + 1, 1ull) == (unsigned long long)gridDim.x - 1) {
+        atomicExch(p.tickets, 0ull);
+        atomicExch(p.tickets + 1, 0ull);
+      }
+      // no copy into this CTA's shared memory may still be in flight at exit
+      if (nkv > 0) mbar_wait(&bars->kv_full, (nkv - 1) & 1, 33);
+      for (int s = 0; s < NST && s < g; ++s) {
+        const int last = s + ((g - 1 - s) / NST) * NST;
         mbar_wait(&bars->q_full[s], (last / NST) & 1, 34);
       }
-      if (do_issued > 0) mbar_wait(&bars->do_full, (do_issued - 1) & 1, 48);
+      if (dog > 0) mbar_wait(&bars->do_full, (dog - 1) & 1, 48);
     }
    } else if (warp == kMmaWarp) {
+    bool ok = true;
+    int g = 0;  // query tiles over all items
+    // One descriptor for the start of shared memory (the K tile, K-major); every
+    // operand is a compile-time offset from it (one add per MMA), a Q stage a
+    // per-tile one, and an MN-major operand differs only in LBO.
+    const uint64_t d0 = sdesc_sw128(smem_u32(smem), 16, 1024);
+    constexpr uint64_t kToMn = (uint64_t)((C::CHUNK >> 4) - 1) << 16;  // LBO 16 B -> CHUNK
+    auto q_desc = [&](int gt) { return sdesc_at(opaque(d0), C::OFF_Q + (gt % NST) * C::TILE); };
+    // S^T = K Q^T  (keys x queries), K = d
+    auto issue_s = [&](int gt) {
+      const uint64_t dq = q_desc(gt), dk = opaque(d0);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+        mma_ss(tmem + C::T_S, sdesc_at(dk, C::OFF_K + ko), sdesc_at(dq, ko), C::IDESC_S, kk > 0);
+      }
+      mma_commit(&bars->s_full);
+    };
+    // dP^T = V dO^T
+    auto issue_dp = [&]() {
+      const uint64_t d = opaque(d0);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+        mma_ss(tmem + C::T_DP, sdesc_at(d, C::OFF_V + ko), sdesc_at(d, C::OFF_DO + ko), C::IDESC_S,
+               kk > 0);
+      }
+      mma_commit(&bars->dp_full);
+    };
+    // dV += P^T dO  (keys x d), K = 128 queries, P^T from tensor memory (queries
+    // 64h .. 64h+63 packed at column 64h); the item's first tile starts the sum
+    auto issue_dv = [&](bool first) {
+      const uint64_t d = opaque(d0) + kToMn;
+#pragma unroll
+      for (int kk = 0; kk < BM / 16; ++kk)
+        mma_ts(tmem + C::T_DV, tmem + C::T_S + 64 * (kk / 4) + 8 * (kk % 4),
+               sdesc_at(d, C::OFF_DO + kk * 2048), C::IDESC_DKV, (!first || kk > 0) ? 1u : 0u);
+      mma_commit(&bars->do_empty);
+    };
+    // Order per item: S(0), dP(0), then per query tile i
+    //   dV(i) | S(i+1) | dQ(i) | dK(i) | dP(i+1)
+    // S(i+1) is issued as soon as dV(i) has read P^T(i) from the S columns (the
+    // compute warps no longer touch them in tile i), so it runs while they form
+    // dS(i); dQ(i) and dK(i) then run while they form P(i+1).  The next item's
+    // S(0) follows the last dK in issue order; its dP(0) waits, like every dP,
+    // until the dQ drawn from the same columns has been drained.
+    for (int r = 0; ok; ++r) {
+      int item = p.items;
+      ok = take_item(r, item, 52);
+      if (!ok || item >= p.items) break;
+      const Item w = decode_item(p, item);
+      if (lane == 0) {
+        ok = mbar_wait(&bars->kv_full, r & 1, 35);
+        if (ok) ok = mbar_wait(&bars->q_full[g % NST], (g / NST) & 1, 36);
+        if (ok) {
+          tc_fence_after();
+          issue_s(g);
+          if (kDQ && g > 0) ok = mbar_wait(&bars->dq_empty, (g - 1) & 1, 37);
+        }
+        if (ok) ok = mbar_wait(&bars->do_full, g & 1, 49);
+        if (ok) {
+          tc_fence_after();
+          issue_dp();
+        }
+        for (int it = 0; it < w.niter && ok; ++it, ++g) {
+          const int st = g % NST;
+          const bool more = it + 1 < w.niter;
+          ok = mbar_wait(&bars->p_full, g & 1, 46);
+          if (!ok) break;
+          tc_fence_after();
+          issue_dv(it == 0);
+          if (!kDQ && !more) mma_commit(&bars->kv_empty);  // the item's last reads of K and V are issued
+          if (more) {
+            ok = mbar_wait(&bars->q_full[(g + 1) % NST], ((g + 1) / NST) & 1, 36);
+            if (!ok) break;
+            tc_fence_after();
+            issue_s(g + 1);
+          }
+          ok = mbar_wait(&bars->ds_full, g & 1, 38);
+          if (!ok) break;
+          tc_fence_after();
+          if constexpr (kDQ) {
+            // dQ_part = dS K  (queries x d), K = 128 keys; written over dP^T
+            const uint64_t dmn = opaque(d0) + kToMn;
+#pragma unroll
+            for (int kk = 0; kk < BN / 16; ++kk)
+              mma_ss(tmem + C::T_DP, sdesc_at(dmn, C::OFF_DS + kk * 2048), sdesc_at(dmn, C::OFF_K + kk * 2048),
+                     C::IDESC_DQ, kk > 0);
+            mma_commit(&bars->dq_full);
+            if (!more) mma_commit(&bars->kv_empty);
+          }
+          // dK += dS^T Q  (keys x d), K = 128 queries
+          const uint64_t dq_mn = q_desc(g) + kToMn, dds = opaque(d0);
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk) {
+            const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+            mma_ss(tmem + C::T_DK, sdesc_at(dds, C::OFF_DS + ko), sdesc_at(dq_mn, kk * 2048), C::IDESC_DKV,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bars->ds_free);
+          mma_commit(&bars->q_empty[st]);
+          if (!more) mma_commit(&bars->acc_full);  // dK, dV of the item complete
+          if (more) {
+            // dP^T(i+1) overwrites the columns dQ(i) was drained from; without dQ
+            // the compute warps have read dP^T(i) before they published dS(i)
+            if constexpr (kDQ) ok = mbar_wait(&bars->dq_empty, g & 1, 37);
+            if (ok) ok = mbar_wait(&bars->do_full, (g + 1) & 1, 49);
+            if (!ok) break;
+            tc_fence_after();
+            issue_dp();
+          }
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      g = __shfl_sync(0xffffffffu, g, 0);
+    }
     if (lane == 0) {
-      // One descriptor for the start of shared memory (the K tile, K-major); every
-      // operand is a compile-time offset from it (one add per MMA), a Q stage a
-      // per-tile one, and an MN-major operand differs only in LBO.
-      const uint64_t d0 = sdesc_sw128(smem_u32(smem), 16, 1024);
-      constexpr uint64_t kToMn = (uint64_t)((C::CHUNK >> 4) - 1) << 16;  // LBO 16 B -> CHUNK
-      auto q_desc = [&](int it) { return sdesc_at(opaque(d0), C::OFF_Q + (it % NST) * C::TILE); };
-      // S^T = K Q^T  (keys x queries), K = d
-      auto issue_s = [&](int it) {
-        const uint64_t dq = q_desc(it), dk = opaque(d0);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_ss(tmem + C::T_S, sdesc_at(dk, C::OFF_K + ko), sdesc_at(dq, ko), C::IDESC_S, kk > 0);
-        }
-        mma_commit(&bars->s_full);
-      };
-      // dP^T = V dO^T
-      auto issue_dp = [&](int it) {
-        const uint64_t d = opaque(d0);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_ss(tmem + C::T_DP, sdesc_at(d, C::OFF_V + ko), sdesc_at(d, C::OFF_DO + ko), C::IDESC_S,
-                 kk > 0);
-        }
-        mma_commit(&bars->dp_full);
-      };
-      // dV += P^T dO  (keys x d), K = 128 queries, P^T from tensor memory (queries
-      // 64h .. 64h+63 packed at column 64h)
-      auto issue_dv = [&](int it) {
-        const uint64_t d = opaque(d0) + kToMn;
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ts(tmem + C::T_DV, tmem + C::T_S + 64 * (kk / 4) + 8 * (kk % 4),
-                 sdesc_at(d, C::OFF_DO + kk * 2048), C::IDESC_DKV, (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&bars->do_empty);
-      };
-      // Order per query tile i (after the prologue S(0), dP(0)):
-      //   dV(i) | S(i+1) | dQ(i) | dK(i) | dP(i+1)
-      // S(i+1) is issued as soon as dV(i) has read P^T(i) from the S columns (the
-      // compute warps no longer touch them in tile i), so it runs while they form
-      // dS(i); dQ(i) and dK(i) then run while they form P(i+1).
-      bool ok = mbar_wait(&bars->kv_full, 0, 35);
-      if (ok) ok = mbar_wait(&bars->q_full[0], 0, 36);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
-        ok = mbar_wait(&bars->do_full, 0, 49);
-      }
-      if (ok) {
-        tc_fence_after();
-        issue_dp(0);
-      }
-      for (int it = 0; it < niter && ok; ++it) {
-        const int st = it % NST;
-        const bool more = it + 1 < niter;
-        ok = mbar_wait(&bars->p_full, it & 1, 46);
-        if (!ok) break;
-        tc_fence_after();
-        issue_dv(it);
-        if (more) {
-          ok = mbar_wait(&bars->q_full[(it + 1) % NST], ((it + 1) / NST) & 1, 36);
-          if (!ok) break;
-          tc_fence_after();
-          issue_s(it + 1);
-        }
-        ok = mbar_wait(&bars->ds_full, it & 1, 38);
-        if (!ok) break;
-        tc_fence_after();
-        if constexpr (kDQ) {
-          // dQ_part = dS K  (queries x d), K = 128 keys; written over dP^T
-          const uint64_t dmn = opaque(d0) + kToMn;
-#pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk)
-            mma_ss(tmem + C::T_DP, sdesc_at(dmn, C::OFF_DS + kk * 2048), sdesc_at(dmn, C::OFF_K + kk * 2048),
-                   C::IDESC_DQ, kk > 0);
-          mma_commit(&bars->dq_full);
-        }
-        // dK += dS^T Q  (keys x d), K = 128 queries
-        const uint64_t dq_mn = q_desc(it) + kToMn, dds = opaque(d0);
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-          mma_ss(tmem + C::T_DK, sdesc_at(dds, C::OFF_DS + ko), sdesc_at(dq_mn, kk * 2048), C::IDESC_DKV,
-                 (it > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&bars->ds_free);
-        mma_commit(&bars->q_empty[st]);
-        if (more) {
-          // dP^T(i+1) overwrites the columns dQ(i) was drained from; without dQ
-          // the compute warps have read dP^T(i) before they published dS(i)
-          if constexpr (kDQ) ok = mbar_wait(&bars->dq_empty, it & 1, 37);
-          if (ok) ok = mbar_wait(&bars->do_full, (it + 1) & 1, 49);
-          if (!ok) break;
-          tc_fence_after();
-          issue_dp(it + 1);
-        }
-      }
-      if (ok) mma_commit(&bars->all_done);
       mma_commit(&bars->drain);
       mbar_wait(&bars->drain, 0, 39);
     }
-   }
+    __syncwarp();
+  } 
   } else if (warp < 8) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsCompute));
     // Compute warps 0-7.  Warp w owns tensor-memory lane quarter w % 4 (key rows
     // 32*(w%4) .. +31 for S^T/dP^T/dK/dV) and column half h = w / 4: query
     // columns 64h .. 64h+63 of P^T and dS, dK / dV columns (d/2)h .. +d/2-1.  Per
-    // query tile: P^T -> tensor memory, dS -> shared memory.
+    // query tile: P^T -> tensor memory, dS -> shared memory; per item: dK, dV.
     const int qw = warp % 4, h = warp / 4;
     const int r = qw * 32 + lane;
-    const int kr = j * BN + r;
-    const bool key_ok = kr < p.Nk;
     const uint32_t lane_off = (uint32_t)(qw * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::T_S;
     const uint32_t tDP = tmem + lane_off + C::T_DP;
     const float c = p.scale_log2;
     const uint32_t ds_row = smem_u32(sDS) + h * C::CHUNK + r * 128;
-    constexpr int DH = D / 2;  // dQ / dK / dV columns per warp
     bool ok = true;
-    for (int it = 0; it < niter && ok; ++it) {
-      const int i = q_tile(it), st = it % NST;
-      const uint32_t lse2 = smem_u32(sVec + st * 2 * BM) + h * 64 * 4;  // -LSE*log2(e), my columns
-      const uint32_t dsv = lse2 + BM * 4;                                // -D, my columns
-      ok = mbar_wait(&bars->q_full[st], (it / NST) & 1, 40);
-      if (ok) ok = mbar_wait(&bars->s_full, it & 1, 41);
-      if (!ok) break;
-      tc_fence_after();
-      float pr[64];
+    int g = 0;
+    for (int ri = 0; ok; ++ri) {
+      int item = p.items;
+      ok = take_item(ri, item, 53);
+      if (!ok || item >= p.items) break;
+      const Item w = decode_item(p, item);
+      const int kr = w.j * BN + r;
+      const bool key_ok = kr < p.Nk;
+      for (int it = 0; it < w.niter && ok; ++it, ++g) {
+        const int i = w.i0 + it % w.nqi, st = g % NST;
+        const uint32_t lse2 = smem_u32(sVec + st * 2 * BM) + h * 64 * 4;  // -LSE*log2(e), my columns
+        const uint32_t dsv = lse2 + BM * 4;                                // -D, my columns
+        ok = mbar_wait(&bars->q_full[st], (g / NST) & 1, 40);
+        if (ok) ok = mbar_wait(&bars->s_full, g & 1, 41);
+        if (!ok) break;
+        tc_fence_after();
+        float pr[64];
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tS + h * 64 + cc * 32, v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) pr[cc * 32 + e] = __uint_as_float(v[e]);
-      }
-      tmem_wait_ld();
-      // Masked keys get S = -inf before the exponentials (P = 0): key j*BN + r is
-      // hidden from query i*BM + 64h + col iff col < hide (above the causal
-      // diagonal), and from every query if it is past Nk.
-      {
-        const int hide = !key_ok ? 64 : p.causal ? min(max(r + (j - i) * BN - p.off - h * 64, 0), 64) : 0;
-        if (hide > 0) {
-#pragma unroll
-          for (int col = 0; col < 64; ++col)
-            if (col < hide) pr[col] = -INFINITY;
-        }
-      }
-      const uint64_t c2 = f2_pack(c, c);
-#pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 l4 = ld_shared_v4(lse2 + c4 * 16);
-        // x = s * c - LSE * log2(e) for two columns at a time (the vector holds -LSE * log2(e))
-        float x0, x1, x2, x3;
-        f2_unpack(f2_fma(f2_pack(pr[4 * c4], pr[4 * c4 + 1]), c2, f2_pack(l4.x, l4.y)), x0, x1);
-        f2_unpack(f2_fma(f2_pack(pr[4 * c4 + 2], pr[4 * c4 + 3]), c2, f2_pack(l4.z, l4.w)), x2, x3);
-        pr[4 * c4] = ex2(x0);
-        pr[4 * c4 + 1] = ex2(x1);
-        pr[4 * c4 + 2] = ex2(x2);
-        pr[4 * c4 + 3] = ex2(x3);
-      }
-      {
-        uint32_t v[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
-        // packed P^T of my 64 query columns over the first 32 of my own S columns
-        tmem_st32(tS + h * 64, v);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars->p_full);
-      ok = mbar_wait(&bars->dp_full, it & 1, 42);
-      if (ok && it > 0) ok = mbar_wait(&bars->ds_free, (it - 1) & 1, 43);
-      if (!ok) break;
-      tc_fence_after();
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t v[32];
-        tmem_ld32(tDP + h * 64 + cc * 32, v);
-        tmem_wait_ld();
-        uint32_t w[16];
-#pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const int c0 = cc * 32 + 4 * e4;
-          const float4 dd = ld_shared_v4(dsv + c0 * 4);
-          // dS = P * (dP - D), two columns per packed instruction (the vector holds -D)
-          float d0, d1, d2, d3;
-          f2_unpack(f2_mul(f2_pack(pr[c0], pr[c0 + 1]),
-                           f2_add(f2_pack(__uint_as_float(v[4 * e4]), __uint_as_float(v[4 * e4 + 1])),
-                                  f2_pack(dd.x, dd.y))), d0, d1);
-          f2_unpack(f2_mul(f2_pack(pr[c0 + 2], pr[c0 + 3]),
-                           f2_add(f2_pack(__uint_as_float(v[4 * e4 + 2]), __uint_as_float(v[4 * e4 + 3])),
-                                  f2_pack(dd.z, dd.w))), d2, d3);
-          w[2 * e4] = pack_bf16x2(d0, d1);
-          w[2 * e4 + 1] = pack_bf16x2(d2, d3);
-        }
-        // row r of the dS^T tile in the 128-byte swizzled layout: chunk h,
-        // 16-byte units cc*4 .. cc*4+3 XOR (r % 8)
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const uint32_t unit = (uint32_t)(cc * 4 + u) ^ (uint32_t)(r & 7);
-          st_shared_v4(ds_row + unit * 16, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(&bars->ds_full);
-    }
-    if (ok) ok = mbar_wait(&bars->all_done, 0, 44);
-    if (ok) {
-      tc_fence_after();
-      const size_t row = (size_t)bkv * p.Nk + (size_t)(key_ok ? kr : 0);
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t tsrc = tmem + lane_off + (which ? C::T_DV : C::T_DK) + h * DH;
-        __nv_bfloat16* dst = (which ? p.dv : p.dk) + row * D + h * DH;
-        const float mul = which ? 1.f : p.scale;
-#pragma unroll
-        for (int cc = 0; cc < DH / 32; ++cc) {
+        for (int cc = 0; cc < 2; ++cc) {
           uint32_t v[32];
-          tmem_ld32(tsrc + cc * 32, v);
+          tmem_ld32(tS + h * 64 + cc * 32, v);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pr[cc * 32 + e] = __uint_as_float(v[e]);
+        }
+        tmem_wait_ld();
+        // Masked keys get S = -inf before the exponentials (P = 0): key j*BN + r is
+        // hidden from query i*BM + 64h + col iff col < hide (above the causal
+        // diagonal), and from every query if it is past Nk.
+        {
+          const int hide = !key_ok ? 64 : p.causal ? min(max(r + (w.j - i) * BN - p.off - h * 64, 0), 64) : 0;
+          if (hide > 0) {
+#pragma unroll
+            for (int col = 0; col < 64; ++col)
+              if (col < hide) pr[col] = -INFINITY;
+          }
+        }
+        const uint64_t c2 = f2_pack(c, c);
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 l4 = ld_shared_v4(lse2 + c4 * 16);
+          // x = s * c - LSE * log2(e) for two columns at a time (the vector holds -LSE * log2(e))
+          float x0, x1, x2, x3;
+          f2_unpack(f2_fma(f2_pack(pr[4 * c4], pr[4 * c4 + 1]), c2, f2_pack(l4.x, l4.y)), x0, x1);
+          f2_unpack(f2_fma(f2_pack(pr[4 * c4 + 2], pr[4 * c4 + 3]), c2, f2_pack(l4.z, l4.w)), x2, x3);
+          pr[4 * c4] = ex2(x0);
+          pr[4 * c4 + 1] = ex2(x1);
+          pr[4 * c4 + 2] = ex2(x2);
+          pr[4 * c4 + 3] = ex2(x3);
+        }
+        {
+          uint32_t v[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = pack_bf16x2(pr[2 * e], pr[2 * e + 1]);
+          // packed P^T of my 64 query columns over the first 32 of my own S columns
+          tmem_st32(tS + h * 64, v);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full);
+        ok = mbar_wait(&bars->dp_full, g & 1, 42);
+        if (ok && g > 0) ok = mbar_wait(&bars->ds_free, (g - 1) & 1, 43);
+        if (!ok) break;
+        if (it == 0 && ri > 0) {
+          // this warp's dK / dV stores of the previous item must have read its
+          // part of the dS buffer
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          __syncwarp();
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tDP + h * 64 + cc * 32, v);
           tmem_wait_ld();
-          if (key_ok) {
-            uint32_t w[16];
+          uint32_t wv[16];
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const int c0 = cc * 32 + 4 * e4;
+            const float4 dd = ld_shared_v4(dsv + c0 * 4);
+            // dS = P * (dP - D), two columns per packed instruction (the vector holds -D)
+            float d0, d1, d2, d3;
+            f2_unpack(f2_mul(f2_pack(pr[c0], pr[c0 + 1]),
+                             f2_add(f2_pack(__uint_as_float(v[4 * e4]), __uint_as_float(v[4 * e4 + 1])),
+                                    f2_pack(dd.x, dd.y))), d0, d1);
+            f2_unpack(f2_mul(f2_pack(pr[c0 + 2], pr[c0 + 3]),
+                             f2_add(f2_pack(__uint_as_float(v[4 * e4 + 2]), __uint_as_float(v[4 * e4 + 3])),
+                                    f2_pack(dd.z, dd.w))), d2, d3);
+            wv[2 * e4] = pack_bf16x2(d0, d1);
+            wv[2 * e4 + 1] = pack_bf16x2(d2, d3);
+          }
+          // row r of the dS^T tile in the 128-byte swizzled layout: chunk h,
+          // 16-byte units cc*4 .. cc*4+3 XOR (r % 8)
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t unit = (uint32_t)(cc * 4 + u) ^ (uint32_t)(r & 7);
+            st_shared_v4(ds_row + unit * 16, wv[4 * u], wv[4 * u + 1], wv[4 * u + 2], wv[4 * u + 3]);
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bars->ds_full);
+      }
+      // dK, dV of the item: tensor memory -> bf16 rows.  The next item's first
+      // dV and dK overwrite these columns only after this warp has published that
+      // item's first P and dS, i.e. after the loads below have completed.
+      if (ok) ok = mbar_wait(&bars->acc_full, ri & 1, 44);
+      if (!ok) break;
+      tc_fence_after();
+      // dK, dV of the item: tensor memory -> bf16 -> this warp's 32 x 128-byte
+      // part of the dS buffer (the part it writes dS to; the item's last dK and
+      // dQ GEMMs have read it) in the 128-byte-swizzled layout -> one TMA store
+      // of a 32-row box by lane 0.  Warp (qw, h) stores rows 32qw .. 32qw+31:
+      // at d = 128 columns 64h .. 64h+63 of dV, then of dK; at d = 64 all
+      // columns of dV (h = 0) or dK (h = 1).  Rows past Nk are clipped by the
+      // tensor map, and a box that starts past Nk is not stored.
+      {
+        constexpr int NT = D == 128 ? 2 : 1;
+        const uint32_t region = smem_u32(sDS) + h * C::CHUNK + qw * 32 * 128;
+        const int row0 = w.j * BN + qw * 32;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const bool isK = D == 128 ? (t == 1) : (h == 1);
+          const uint32_t tsrc = tmem + lane_off + (isK ? C::T_DK : C::T_DV) + (D == 128 ? h * 64 : 0);
+          const float mul = isK ? p.scale : 1.f;
+          uint32_t wv[32];
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(tsrc + cc * 32, v);
+            tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 16; ++e)
-              w[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
-            uint4* o4 = reinterpret_cast<uint4*>(dst + cc * 32);
+              wv[cc * 16 + e] = pack_bf16x2(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+          }
+          if (t > 0) {
+            // the store of the first tensor must have read the region
+            if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            __syncwarp();
+          }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) o4[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+          for (int u = 0; u < 8; ++u)
+            st_shared_v4(region + lane * 128 + ((u ^ (lane & 7)) << 4), wv[4 * u], wv[4 * u + 1], wv[4 * u + 2],
+                         wv[4 * u + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (row0 < p.Nk) tma_store_3d(isK ? &mdk : &mdv, region, D == 128 ? h * 64 : 0, row0, w.bkv);
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
           }
         }
       }
+      tc_fence_before();
     }
+    // no store may still be reading this CTA's shared memory at exit
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    __syncwarp();
   } else if constexpr (!kDQ) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsReduce));
   } else {
@@ -527,36 +683,42 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tQ = tmem + ((uint32_t)(qw * 32) << 16) + C::T_DP;
     const uint32_t stg0 = smem_u32(smem + C::OFF_STG + qw * 2 * C::STG_BYTES);
     bool ok = true;
-    int chunk = 0;
-    for (int it = 0; it < niter && ok; ++it) {
-      ok = mbar_wait(&bars->dq_full, it & 1, 45);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t v[D / 32][32];
+    int chunk = 0, g = 0;
+    for (int ri = 0; ok; ++ri) {
+      int item = p.items;
+      ok = take_item(ri, item, 54);
+      if (!ok || item >= p.items) break;
+      const Item w = decode_item(p, item);
+      for (int it = 0; it < w.niter && ok; ++it, ++g) {
+        ok = mbar_wait(&bars->dq_full, g & 1, 45);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t v[D / 32][32];
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tQ + cc * 32, v[cc]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bars->dq_empty);
-      const int row0 = q_tile(it) * BM + qw * 32, bh = q_head(it);
+        for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tQ + cc * 32, v[cc]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->dq_empty);
+        const int row0 = (w.i0 + it % w.nqi) * BM + qw * 32, bh = w.bhq0 + it / w.nqi;
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc, ++chunk) {
-        const uint32_t buf = stg0 + (chunk & 1) * C::STG_BYTES;
-        if (chunk >= 2) {
-          // the reduce that read this buffer two chunks ago must be done with it
-          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+        for (int cc = 0; cc < D / 32; ++cc, ++chunk) {
+          const uint32_t buf = stg0 + (chunk & 1) * C::STG_BYTES;
+          if (chunk >= 2) {
+            // the reduce that read this buffer two chunks ago must be done with it
+            if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+            __syncwarp();
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            st_shared_v4(buf + lane * 128 + ((u ^ (lane & 7)) << 4), v[cc][4 * u], v[cc][4 * u + 1],
+                         v[cc][4 * u + 2], v[cc][4 * u + 3]);
+          fence_proxy_async_smem();
           __syncwarp();
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          st_shared_v4(buf + lane * 128 + ((u ^ (lane & 7)) << 4), v[cc][4 * u], v[cc][4 * u + 1],
-                       v[cc][4 * u + 2], v[cc][4 * u + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          // rows past N are clipped by the tensor map; a box wholly past N is skipped
-          if (row0 < p.Nq) tma_reduce_add_3d(&mdq, buf, cc * 32, row0, bh);
-          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          if (lane == 0) {
+            // rows past N are clipped by the tensor map; a box wholly past N is skipped
+            if (row0 < p.Nq) tma_reduce_add_3d(&mdq, buf, cc * 32, row0, bh);
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          }
         }
       }
     }
@@ -584,9 +746,11 @@ __global__ void __launch_bounds__(256) preprocess_kernel(const __nv_bfloat16* __
                                                          const float* __restrict__ lse,
                                                          float* __restrict__ lse2,
                                                          float* __restrict__ dsum,
-                                                         float* __restrict__ dq_acc, int BH, int N,
-                                                         int Npad) {
+                                                         float* __restrict__ dq_acc,
+                                                         unsigned long long* __restrict__ tickets,
+                                                         int BH, int N, int Npad) {
   constexpr int L = D / 8;          // lanes per row
+  if (blockIdx.x == 0 && threadIdx.x < 2) tickets[threadIdx.x] = 0ull;  // the main kernel's scheduler
   constexpr int RPW = 32 / L;       // rows per warp
   const int lane = threadIdx.x % 32;
   const long long gr = ((long long)blockIdx.x * 8 + threadIdx.x / 32) * RPW + lane / L;
@@ -1050,7 +1214,7 @@ size_t sm100_backward_workspace(int BH, int N, int d) {
   const size_t npad = (size_t)(N + 127) / 128 * 128;
   const size_t vec = ((size_t)BH * npad * 4 + 255) / 256 * 256;
   const size_t acc = ((size_t)BH * N * d * 4 + 255) / 256 * 256;
-  return 2 * vec + acc;
+  return 2 * vec + acc + 256;  // + the main kernel's two ticket counters
 }
 
 size_t sm100_backward_dq_offset(int BH, int N) {
@@ -1062,13 +1226,13 @@ namespace {
 
 template <int D, bool kDQ>
 cudaError_t launch_main(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                        const CUtensorMap& mdo, const CUtensorMap& mdq, const bwd::Params& p,
-                        cudaStream_t st) {
+                        const CUtensorMap& mdo, const CUtensorMap& mdq, const CUtensorMap& mdk,
+                        const CUtensorMap& mdv, const bwd::Params& p, cudaStream_t st) {
   const int smem = bwd::Cfg<D>::SMEM_BYTES;
   cudaError_t e = cudaFuncSetAttribute(bwd::main_kernel<D, kDQ>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  bwd::main_kernel<D, kDQ><<<grid, bwd::NTHREADS, smem, st>>>(mq, mk, mv, mdo, mdq, p);
+  bwd::main_kernel<D, kDQ><<<grid, bwd::NTHREADS, smem, st>>>(mq, mk, mv, mdo, mdq, mdk, mdv, p);
   return cudaGetLastError();
 }
 
@@ -1086,7 +1250,8 @@ cudaError_t launch_dq(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, c
 }  // namespace
 
 cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                           const CUtensorMap& mdo, const CUtensorMap& mdq, const void* o,
+                           const CUtensorMap& mdo, const CUtensorMap& mdq, const CUtensorMap& mdk,
+                           const CUtensorMap& mdv, const void* o,
                            const void* dout, const float* lse,
                            void* dq, void* dk, void* dv, void* workspace, int B, int H, int Hkv,
                            int Nq, int Nk, int d, float scale, int causal, int stages,
@@ -1099,6 +1264,8 @@ cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const C
   float* lse2 = static_cast<float*>(workspace);
   float* dsum = reinterpret_cast<float*>(static_cast<char*>(workspace) + vec);
   float* acc = reinterpret_cast<float*>(static_cast<char*>(workspace) + 2 * vec);
+  auto* tickets = reinterpret_cast<unsigned long long*>(
+      static_cast<char*>(workspace) + 2 * vec + ((size_t)BH * N * d * 4 + 255) / 256 * 256);
   cudaError_t e = cudaSuccess;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess)
@@ -1112,14 +1279,14 @@ cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const C
     const auto* gb = static_cast<const __nv_bfloat16*>(dout);
     if (d == 128) {
       if (det)
-        bwd::preprocess_kernel<128, false><<<pblocks, 256, 0, st>>>(ob, gb, lse, lse2, dsum, acc, BH, N, npad);
+        bwd::preprocess_kernel<128, false><<<pblocks, 256, 0, st>>>(ob, gb, lse, lse2, dsum, acc, tickets, BH, N, npad);
       else
-        bwd::preprocess_kernel<128, true><<<pblocks, 256, 0, st>>>(ob, gb, lse, lse2, dsum, acc, BH, N, npad);
+        bwd::preprocess_kernel<128, true><<<pblocks, 256, 0, st>>>(ob, gb, lse, lse2, dsum, acc, tickets, BH, N, npad);
     } else {
       if (det)
-        bwd::preprocess_kernel<64, false><<<pblocks, 256, 0, st>>>(ob, gb, lse, lse2, dsum, acc, BH, N, npad);
+        bwd::preprocess_kernel<64, false><<<pblocks, 256, 0, st>>>(ob, gb, lse, lse2, dsum, acc, tickets, BH, N, npad);
       else
-        bwd::preprocess_kernel<64, true><<<pblocks, 256, 0, st>>>(ob, gb, lse, lse2, dsum, acc, BH, N, npad);
+        bwd::preprocess_kernel<64, true><<<pblocks, 256, 0, st>>>(ob, gb, lse, lse2, dsum, acc, tickets, BH, N, npad);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -1145,13 +1312,16 @@ cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const C
     p.scale_log2 = scale * bwd::kLog2e;
     p.causal = causal;
     p.chunk = bwd::chunk_heads(p.BHkv, p.G, Nq, Nk, d, p.nkv, sms);
-    const dim3 grid((unsigned)(p.nkv * p.BHkv));
+    p.items = p.nkv * p.BHkv;
+    p.tickets = tickets;
+    // persistent: one CTA per SM, each taking items as it becomes free
+    const dim3 grid((unsigned)std::min(p.items, sms));
     if (det)
-      e = d == 128 ? launch_main<128, false>(grid, mq, mk, mv, mdo, mdq, p, st)
-                   : launch_main<64, false>(grid, mq, mk, mv, mdo, mdq, p, st);
+      e = d == 128 ? launch_main<128, false>(grid, mq, mk, mv, mdo, mdq, mdk, mdv, p, st)
+                   : launch_main<64, false>(grid, mq, mk, mv, mdo, mdq, mdk, mdv, p, st);
     else
-      e = d == 128 ? launch_main<128, true>(grid, mq, mk, mv, mdo, mdq, p, st)
-                   : launch_main<64, true>(grid, mq, mk, mv, mdo, mdq, p, st);
+      e = d == 128 ? launch_main<128, true>(grid, mq, mk, mv, mdo, mdq, mdk, mdv, p, st)
+                   : launch_main<64, true>(grid, mq, mk, mv, mdo, mdq, mdk, mdv, p, st);
     if (e != cudaSuccess) return e;
   }
   if (!(stages & kStageConvert)) return cudaSuccess;

@@ -52,8 +52,10 @@ constexpr int kStagePreprocess = 1, kStageMain = 2, kStageConvert = 4, kStageAll
 constexpr int kStageDeterministic = 8;
 // mq, mdo, mdq over Nq rows; mk, mv over Nk rows.
 // mdq: 3-D fp32 view {d, Nq, B*H} of the accumulator, box {32, 32, 1}, 128-byte swizzle
+// mdk, mdv: bf16 views {d, Nk, B*Hkv} of dK and dV, box {64, 32, 1}, 128-byte swizzle
 cudaError_t sm100_backward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                           const CUtensorMap& mdo, const CUtensorMap& mdq, const void* o,
+                           const CUtensorMap& mdo, const CUtensorMap& mdq, const CUtensorMap& mdk,
+                           const CUtensorMap& mdv, const void* o,
                            const void* dout, const float* lse,
                            void* dq, void* dk, void* dv, void* workspace, int B, int H, int Hkv,
                            int Nq, int Nk, int d, float scale, int causal, int stages,

@@ -117,7 +117,9 @@ fa_status fa_forward_fp32(const float* q, const float* k, const float* v, float*
 
 /* Bytes of device scratch fa_backward needs for this shape (0 on bad sizes):
  * -LSE*log2(e) and -D_i = -sum_c dO[i,c] * O[i,c] padded to whole 128-row tiles
- * (fp32, [B,H,Npad]) and an fp32 dQ accumulator ([B,H,N,d]). */
+ * (fp32, [B,H,Npad]), an fp32 dQ accumulator ([B,H,N,d]) and 256 bytes for the
+ * work-item counters of the persistent main kernel, each segment rounded up to
+ * 256 bytes. */
 size_t fa_backward_workspace_size(int B, int H, int N, int d);
 
 /* Backward pass, bf16 storage, fp32 accumulation.

@@ -71,16 +71,16 @@ def test_forward_rejects_bad_arguments(lib, fn):
 
 
 def test_workspace_size(lib):
-    # LSE*log2(e) and D padded to 128-row tiles, plus an fp32 dQ accumulator,
-    # each segment rounded up to 256 bytes
+    # LSE*log2(e) and D padded to 128-row tiles, an fp32 dQ accumulator and the
+    # main kernel's work-item counters, each segment rounded up to 256 bytes
     def expect(B, H, N, d):
         up = lambda x: (x + 255) // 256 * 256
         npad = (N + 127) // 128 * 128
-        return 2 * up(B * H * npad * 4) + up(B * H * N * d * 4)
+        return 2 * up(B * H * npad * 4) + up(B * H * N * d * 4) + 256
 
     assert lib.fa_backward_workspace_size(2, 16, 2048, 128) == expect(2, 16, 2048, 128)
-    assert lib.fa_backward_workspace_size(2, 16, 2048, 128) == 2 * 32 * 2048 * 4 + 32 * 2048 * 128 * 4
-    assert lib.fa_backward_workspace_size(1, 1, 3, 64) == expect(1, 1, 3, 64) == 512 + 512 + 768
+    assert lib.fa_backward_workspace_size(2, 16, 2048, 128) == 2 * 32 * 2048 * 4 + 32 * 2048 * 128 * 4 + 256
+    assert lib.fa_backward_workspace_size(1, 1, 3, 64) == expect(1, 1, 3, 64) == 512 + 512 + 768 + 256
     assert lib.fa_backward_workspace_size(1, 1, 3, 96) == 0
     assert lib.fa_backward_workspace_size(0, 1, 3, 64) == 0
 

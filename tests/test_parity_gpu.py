@@ -155,11 +155,12 @@ def test_backward_fp32_storage():
 @pytest.mark.parametrize("B,H,Hkv,N,d,causal", [(2, 16, 16, 2048, 128, True), (2, 32, 32, 4096, 128, True),
                                                  (1, 24, 6, 4096, 64, True), (1, 8, 8, 8192, 128, False)])
 def test_backward_schedule_covers_every_tile_once(B, H, Hkv, N, d, causal):
-    # The backward runs its (key/value head, key tile) CTAs in L2-sized head
-    # chunks.  dK and dV of a key tile come from one CTA whatever the order, so
-    # a multi-chunk launch must give them bit for bit as launches of one
-    # key/value head each do; dQ is summed by reduce-adds in an order that
-    # varies, so it is held to fp32 rounding.
+    # The persistent backward hands out its (key/value head, key tile) work
+    # items from a ticket counter, in L2-sized head chunks.  dK and dV of a key
+    # tile come from one item whatever the order or the CTA that takes it, so a
+    # multi-chunk launch must give them bit for bit as launches of one key/value
+    # head each do (an item skipped or taken twice would show); dQ is summed by
+    # reduce-adds in an order that varies, so it is held to fp32 rounding.
     q, k, v, do = (t.cuda() for t in make_inputs(B, H, N, d, seed=23, with_do=True))
     k, v = k[:, :Hkv].contiguous(), v[:, :Hkv].contiguous()
     o, lse = fa.forward_gqa(q, k, v, causal=causal)
@@ -176,6 +177,27 @@ def test_backward_schedule_covers_every_tile_once(B, H, Hkv, N, d, causal):
             rel = float((dq1.float() - dq[qs].float()).norm() / dq1.float().norm())
             assert rel < 1e-3, (b, hk, rel)
     fa.check_device_status()
+
+
+def test_backward_ignores_workspace_contents_and_resets_its_counters():
+    # The workspace's contents are ignored on entry: one filled with 0xFF bytes
+    # (the main kernel's two work-item counters included) gives the dK, dV of a
+    # zeroed one bit for bit, and the main kernel leaves both counters at zero
+    # (its last CTA resets them).  The counters are the last 256-byte segment.
+    B, H, N, d = 1, 8, 1000, 128
+    q, k, v, do = (t.cuda() for t in make_inputs(B, H, N, d, seed=31, with_do=True))
+    o, lse = fa.forward(q, k, v, causal=True)
+    size = fa.workspace_size(B, H, N, d)
+    ref = fa.backward(q, k, v, o, do, lse, causal=True,
+                      workspace=torch.zeros(size, dtype=torch.uint8, device="cuda"))
+    ws = torch.full((size,), 255, dtype=torch.uint8, device="cuda")
+    for _ in range(3):  # the same workspace again and again
+        got = fa.backward(q, k, v, o, do, lse, causal=True, workspace=ws)
+        fa.check_device_status()
+        assert torch.equal(got[1], ref[1]) and torch.equal(got[2], ref[2])
+        rel = float((got[0].float() - ref[0].float()).norm() / ref[0].float().norm())
+        assert rel < 1e-3, rel
+        assert ws[size - 256:size - 240].view(torch.int64).tolist() == [0, 0]
 
 
 # ---------------------------------------------------------------- grouped-query
