@@ -157,11 +157,11 @@ fa_status forward_bf16(const void* q, const void* k, const void* v, void* o, flo
   if (Hkv <= 0 || H % Hkv != 0) return FA_ERR_INVALID_ARG;
   if ((s = check_ptrs({q, k, v, o, lse})) != FA_OK) return s;
   if ((s = check_device()) != FA_OK) return s;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_map(&mq, q, d, Nq, B * H) || !make_map(&mk, k, d, Nk, B * Hkv) ||
-      !make_map(&mv, v, d, Nk, B * Hkv))
+      !make_map(&mv, v, d, Nk, B * Hkv) || !make_map(&mo, o, d, Nq, B * H, 32))
     return map_failed();
-  return from_cuda(sm100_forward(mq, mk, mv, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal ? 1 : 0,
+  return from_cuda(sm100_forward(mq, mk, mv, mo, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal ? 1 : 0,
                                  false, 1.0f, 1.0f, static_cast<cudaStream_t>(stream)));
 }
 
@@ -178,11 +178,11 @@ fa_status forward_fp8(const void* q, const void* k, const void* v, void* o, floa
     return FA_ERR_INVALID_ARG;
   if ((s = check_ptrs({q, k, v, o, lse})) != FA_OK) return s;
   if ((s = check_device()) != FA_OK) return s;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_map_fp8(&mq, q, d, Nq, B * H) || !make_map_fp8(&mk, k, d, Nk, B * Hkv) ||
-      !make_map_fp8(&mv, v, d, Nk, B * Hkv))
+      !make_map_fp8(&mv, v, d, Nk, B * Hkv) || !make_map(&mo, o, d, Nq, B * H, 32))
     return map_failed();
-  return from_cuda(sm100_forward(mq, mk, mv, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal ? 1 : 0,
+  return from_cuda(sm100_forward(mq, mk, mv, mo, o, lse, B, H, Hkv, Nq, Nk, d, scale, causal ? 1 : 0,
                                  true, qk, v_descale, static_cast<cudaStream_t>(stream)));
 }
 

@@ -13,7 +13,10 @@
 //
 // CTA layout (384 threads, registers rebalanced with setmaxnreg):
 //   warps 0-3  softmax + epilogue for query tile 0 (tensor-memory lanes 0-127)
-//   warps 4-7  softmax + epilogue for query tile 1
+//   warps 4-7  softmax + epilogue for query tile 1 (at d = 64 the epilogue
+//              stages O in shared memory and stores it with TMA, one 32-row box
+//              per warp; at d = 128 shared memory is full and rows are stored
+//              directly)
 //   warp  8    TMA producer: draws the CTA's next work item when it has issued
 //              the loads of the current one, hands it to the other roles through
 //              a two-entry ring, then loads Q tiles and K_j, V_j into a ring of slots
@@ -90,7 +93,12 @@ struct Cfg {
   static constexpr int NSLOT = F8 ? (D == 128 ? 12 : 16) : (D == 128 ? 5 : 10);  // K/V ring slots
   static constexpr int SMEM_Q = NQT * TILE;
   static constexpr int SMEM_RING = NSLOT * TILE;
-  static constexpr int OFF_BAR = SMEM_Q + SMEM_RING;
+  // At d = 64 shared memory has room to stage O: each softmax warp converts its
+  // 32 rows (128 bytes each) there and stores them with one TMA store.
+  static constexpr bool O_STAGED = D == 64;
+  static constexpr int OFF_O = SMEM_Q + SMEM_RING;
+  static constexpr int SMEM_O = O_STAGED ? NQT * BM * 128 : 0;
+  static constexpr int OFF_BAR = OFF_O + SMEM_O;
   static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;  // barriers + alignment slack
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t IDESC_QK = F8 ? idesc_e4m3(BM, BN, 0, 0) : idesc_bf16(BM, BN, 0, 0);
@@ -184,7 +192,8 @@ __device__ __forceinline__ void decode_item(const Params& p, int item, int& bh, 
 template <int D, bool F8>
 __global__ void __launch_bounds__(NTHREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-               const __grid_constant__ CUtensorMap mv, const Params p) {
+               const __grid_constant__ CUtensorMap mv, const __grid_constant__ CUtensorMap mo,
+               const Params p) {
   using C = Cfg<D, F8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -240,6 +249,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tma_prefetch_desc(&mq);
     tma_prefetch_desc(&mk);
     tma_prefetch_desc(&mv);
+    if (C::O_STAGED) tma_prefetch_desc(&mo);
   }
   tc_fence_before();
   __syncthreads();
@@ -586,6 +596,36 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (ok) {
       tc_fence_after();
       const float inv = l > 0.f ? p.o_scale / l : 0.f;
+      if constexpr (C::O_STAGED) {
+        // rows 32*(warp%4) .. +31 of the tile: bf16 into this warp's 4 KB of the
+        // O staging area (128-byte swizzled), then one TMA store by lane 0; rows
+        // past Nq are clipped by the tensor map, a box starting past Nq skipped
+        const uint32_t region = smem_u32(smem + C::OFF_O) + t * (BM * 128) + (warp % 4) * 4096;
+        const int row0 = q_tile0 + (warp % 4) * 32;
+        uint32_t wv[32];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t r[32];
+          tmem_ld32(tO + cc * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            wv[cc * 16 + i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+        }
+        // the previous item's store from this region must have read it
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          st_shared_v4(region + lane * 128 + ((u ^ (lane & 7)) << 4), wv[4 * u], wv[4 * u + 1], wv[4 * u + 2],
+                         wv[4 * u + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if (row0 < p.Nq) tma_store_3d(&mo, region, 0, row0, bh);
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+      } else {
       __nv_bfloat16* orow = p.o + ((size_t)bh * p.Nq + (size_t)(q_row < p.Nq ? q_row : 0)) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -602,12 +642,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
         }
       }
+      }
       if (q_row < p.Nq)
         p.lse[(size_t)bh * p.Nq + q_row] = l > 0.f ? m_used * p.scale + logf(l) : -INFINITY;
     }
     gtile += n;
     ++icnt;
     }
+    // no O store may still be reading this CTA's shared memory at exit
+    if (C::O_STAGED && lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -663,19 +707,19 @@ namespace {
 
 template <int D, bool F8>
 cudaError_t launch_fwd(dim3 grid, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const fwd::Params& p, cudaStream_t st) {
+                       const CUtensorMap& mo, const fwd::Params& p, cudaStream_t st) {
   const int smem = fwd::Cfg<D, F8>::SMEM_BYTES;
   cudaError_t e = cudaFuncSetAttribute(fwd::fwd_kernel<D, F8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  fwd::fwd_kernel<D, F8><<<grid, fwd::NTHREADS, smem, st>>>(mq, mk, mv, p);
+  fwd::fwd_kernel<D, F8><<<grid, fwd::NTHREADS, smem, st>>>(mq, mk, mv, mo, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                          void* o, float* lse, int B, int H, int Hkv, int Nq, int Nk, int d,
+                          const CUtensorMap& mo, void* o, float* lse, int B, int H, int Hkv, int Nq, int Nk, int d,
                           float scale, int causal, bool fp8, float qk_descale, float v_descale,
                           cudaStream_t st) {
   const int BH = B * H;
@@ -705,10 +749,10 @@ cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   p.slot = (int)(seq % fwd::kSchedSlots);
   p.tag = (unsigned int)(seq % (unsigned long long)(fwd::kHeldTag - 1u)) + 1u;  // 1 .. kHeldTag-1
   if (fp8)
-    return d == 128 ? launch_fwd<128, true>(grid, mq, mk, mv, p, st)
-                    : launch_fwd<64, true>(grid, mq, mk, mv, p, st);
-  return d == 128 ? launch_fwd<128, false>(grid, mq, mk, mv, p, st)
-                  : launch_fwd<64, false>(grid, mq, mk, mv, p, st);
+    return d == 128 ? launch_fwd<128, true>(grid, mq, mk, mv, mo, p, st)
+                    : launch_fwd<64, true>(grid, mq, mk, mv, mo, p, st);
+  return d == 128 ? launch_fwd<128, false>(grid, mq, mk, mv, mo, p, st)
+                  : launch_fwd<64, false>(grid, mq, mk, mv, mo, p, st);
 }
 
 }  // namespace fa

@@ -23,8 +23,9 @@ cudaError_t simt_backward(bool bf16, const void* q, const void* k, const void* v
 // fp8: Q, K, V are e4m3 (maps of uint8 elements, box {min(d, 128), 128, 1}, swizzle
 // of min(d, 128) bytes); the scores are scale * qk_descale * (Q K^T of the stored
 // values) and O = v_descale * P V / l.  bf16: qk_descale = v_descale = 1.
+// mo: bf16 view {d, Nq, B*H} of O, box {64, 32, 1}, 128-byte swizzle (stores at d = 64)
 cudaError_t sm100_forward(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                          void* o, float* lse, int B, int H, int Hkv, int Nq, int Nk, int d,
+                          const CUtensorMap& mo, void* o, float* lse, int B, int H, int Hkv, int Nq, int Nk, int d,
                           float scale, int causal, bool fp8, float qk_descale, float v_descale,
                           cudaStream_t st);
 
