@@ -392,11 +392,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       mma_commit(&bars->do_empty);
     };
     // Order per item: S(0), dP(0), then per query tile i
-    //   dV(i) | S(i+1) | dQ(i) | dK(i) | dP(i+1)
+    //   dV(i) | S(i+1) | dK(i) | dQ(i) | dP(i+1)
     // S(i+1) is issued as soon as dV(i) has read P^T(i) from the S columns (the
     // compute warps no longer touch them in tile i), so it runs while they form
-    // dS(i); dQ(i) and dK(i) then run while they form P(i+1).  The next item's
-    // S(0) follows the last dK in issue order; its dP(0) waits, like every dP,
+    // dS(i); dK(i) and dQ(i) then run while they form P(i+1), dK first so that
+    // Q(i)'s stage is free for Q(i+2) one GEMM earlier.  The next item's
+    // S(0) follows the last dQ in issue order; its dP(0) waits, like every dP,
     // until the dQ drawn from the same columns has been drained.
     for (int r = 0; ok; ++r) {
       int item = p.items;
@@ -433,6 +434,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           ok = mbar_wait(&bars->ds_full, g & 1, 38);
           if (!ok) break;
           tc_fence_after();
+          // dK += dS^T Q  (keys x d), K = 128 queries; before dQ, so that Q's
+          // stage frees for the tile after next one GEMM earlier
+          const uint64_t dq_mn = q_desc(g) + kToMn, dds = opaque(d0);
+#pragma unroll
+          for (int kk = 0; kk < BM / 16; ++kk) {
+            const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
+            mma_ss(tmem + C::T_DK, sdesc_at(dds, C::OFF_DS + ko), sdesc_at(dq_mn, kk * 2048), C::IDESC_DKV,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&bars->q_empty[st]);
           if constexpr (kDQ) {
             // dQ_part = dS K  (queries x d), K = 128 keys; written over dP^T
             const uint64_t dmn = opaque(d0) + kToMn;
@@ -443,16 +454,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mma_commit(&bars->dq_full);
             if (!more) mma_commit(&bars->kv_empty);
           }
-          // dK += dS^T Q  (keys x d), K = 128 queries
-          const uint64_t dq_mn = q_desc(g) + kToMn, dds = opaque(d0);
-#pragma unroll
-          for (int kk = 0; kk < BM / 16; ++kk) {
-            const uint32_t ko = (kk / 4) * C::CHUNK + (kk % 4) * 32;
-            mma_ss(tmem + C::T_DK, sdesc_at(dds, C::OFF_DS + ko), sdesc_at(dq_mn, kk * 2048), C::IDESC_DKV,
-                   (it > 0 || kk > 0) ? 1u : 0u);
-          }
           mma_commit(&bars->ds_free);
-          mma_commit(&bars->q_empty[st]);
           if (!more) mma_commit(&bars->acc_full);  // dK, dV of the item complete
           if (more) {
             // dP^T(i+1) overwrites the columns dQ(i) was drained from; without dQ
