@@ -13,10 +13,10 @@
 //
 // CTA layout (384 threads, registers rebalanced with setmaxnreg):
 //   warps 0-3  softmax + epilogue for query tile 0 (tensor-memory lanes 0-127)
-//   warps 4-7  softmax + epilogue for query tile 1 (at d = 64 the epilogue
-//              stages O in shared memory and stores it with TMA, one 32-row box
-//              per warp; at d = 128 shared memory is full and rows are stored
-//              directly)
+//   warps 4-7  softmax + epilogue for query tile 1 (the epilogue stages O in
+//              shared memory and stores it with TMA, one 32-row box of 64
+//              columns at a time per warp; e4m3 at d = 128 has no room and
+//              stores rows directly)
 //   warp  8    TMA producer: draws the CTA's next work item when it has issued
 //              the loads of the current one, hands it to the other roles through
 //              a two-entry ring, then loads Q tiles and K_j, V_j into a ring of slots
@@ -90,12 +90,14 @@ struct Cfg {
   static constexpr int S_STEPS = D / KSTEP;             // MMAs per S tile
   static constexpr int PV_STEPS = BN / KSTEP;           // MMAs per P V (all 128 keys)
   static constexpr int PCOLS = BN * EB / 4;             // tensor-memory columns of P
-  static constexpr int NSLOT = F8 ? (D == 128 ? 12 : 16) : (D == 128 ? 5 : 10);  // K/V ring slots
+  static constexpr int NSLOT = F8 ? (D == 128 ? 12 : 16) : (D == 128 ? 4 : 10);  // K/V ring slots
   static constexpr int SMEM_Q = NQT * TILE;
   static constexpr int SMEM_RING = NSLOT * TILE;
-  // At d = 64 shared memory has room to stage O: each softmax warp converts its
-  // 32 rows (128 bytes each) there and stores them with one TMA store.
-  static constexpr bool O_STAGED = D == 64;
+  // O staging, 4 KB per softmax warp: it converts 64 columns of its 32 rows
+  // there and stores them with one TMA store (twice at d = 128).  bf16 at d =
+  // 128 makes room with a 4-slot ring, which measured no slower than 5 slots;
+  // e4m3 at d = 128 has none and stores rows directly.
+  static constexpr bool O_STAGED = !F8 || D == 64;
   static constexpr int OFF_O = SMEM_Q + SMEM_RING;
   static constexpr int SMEM_O = O_STAGED ? NQT * BM * 128 : 0;
   static constexpr int OFF_BAR = OFF_O + SMEM_O;
@@ -602,28 +604,33 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // past Nq are clipped by the tensor map, a box starting past Nq skipped
         const uint32_t region = smem_u32(smem + C::OFF_O) + t * (BM * 128) + (warp % 4) * 4096;
         const int row0 = q_tile0 + (warp % 4) * 32;
-        uint32_t wv[32];
+        // 64 columns (one 128-byte swizzle chunk) per round: one round at d = 64,
+        // two at d = 128 through the same 4 KB
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t r[32];
-          tmem_ld32(tO + cc * 32, r);
-          tmem_wait_ld();
+        for (int ch = 0; ch < D / 64; ++ch) {
+          uint32_t wv[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            wv[cc * 16 + i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-        }
-        // the previous item's store from this region must have read it
-        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-        __syncwarp();
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t r[32];
+            tmem_ld32(tO + ch * 64 + cc * 32, r);
+            tmem_wait_ld();
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
-          st_shared_v4(region + lane * 128 + ((u ^ (lane & 7)) << 4), wv[4 * u], wv[4 * u + 1], wv[4 * u + 2],
-                         wv[4 * u + 3]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if (row0 < p.Nq) tma_store_3d(&mo, region, 0, row0, bh);
-          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            for (int i = 0; i < 16; ++i)
+              wv[cc * 16 + i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+          }
+          // the previous store from this region must have read it
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          __syncwarp();
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            st_shared_v4(region + lane * 128 + ((u ^ (lane & 7)) << 4), wv[4 * u], wv[4 * u + 1], wv[4 * u + 2],
+                           wv[4 * u + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (row0 < p.Nq) tma_store_3d(&mo, region, ch * 64, row0, bh);
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          }
         }
       } else {
       __nv_bfloat16* orow = p.o + ((size_t)bh * p.Nq + (size_t)(q_row < p.Nq ? q_row : 0)) * D;
