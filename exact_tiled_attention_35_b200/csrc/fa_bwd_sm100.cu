@@ -59,11 +59,14 @@ constexpr int kRegsReduce = 144;   // warpgroup 2
 constexpr int kRegsControl = 96;   // warpgroup 3: producer, MMA issuer, two idle warps
 static_assert(128 * (2 * kRegsCompute + kRegsReduce + kRegsControl) <= 512 * 128,
               "register split exceeds the launch allocation");
-constexpr int NST = 2;  // Q / dO stages
+constexpr int kMaxNst = 3;  // Q stages at most (Cfg<D>::NST)
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct Cfg {
+  // Q stages (with the LSE / D rows): two at d = 128, where shared memory is
+  // full; three at d = 64, so Q(i+1) can be loaded one query tile earlier
+  static constexpr int NST = D == 64 ? 3 : 2;
   static constexpr int TILE = BN * D * 2;  // bytes of one 128-row bf16 tile
   static constexpr int CHUNK = BN * 128;   // one 64-column swizzle chunk of a tile
   static constexpr int OFF_K = 0;
@@ -78,6 +81,10 @@ struct Cfg {
   static constexpr int SMEM_BYTES = OFF_BAR + 256;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t T_S = 0, T_DP = 128, T_DV = 256, T_DK = 256 + D;
+  // partial dQ: over dP^T at d = 128 (tensor memory is full), in its own
+  // columns at d = 64, where dP^T(i+1) then need not wait for dQ(i)'s drain
+  static constexpr bool DQ_SHARED = D == 128;
+  static constexpr uint32_t T_DQ = DQ_SHARED ? T_DP : 256 + 2 * D;
   static constexpr uint32_t IDESC_S = idesc_bf16(BN, BM, 0, 0);   // K-major x K-major
   static constexpr uint32_t IDESC_DQ = idesc_bf16(BM, D, 1, 1);   // dS (MN) x K (MN)
   static constexpr uint32_t IDESC_DKV = idesc_bf16(BN, D, 0, 1);  // P^T/dS^T (K) x dO/Q (MN)
@@ -112,8 +119,8 @@ constexpr int kItemRing = 2;  // work items the producer may hand out ahead
 struct Bars {
   uint64_t kv_full;
   uint64_t kv_empty;       // the item's last GEMM reading K or V has completed
-  uint64_t q_full[NST];    // Q tile + LSE2 / D vectors of a stage
-  uint64_t q_empty[NST];
+  uint64_t q_full[kMaxNst];    // Q tile + LSE2 / D vectors of a stage
+  uint64_t q_empty[kMaxNst];
   uint64_t do_full;        // dO tile (single buffer)
   uint64_t do_empty;
   uint64_t s_full;
@@ -216,7 +223,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   uint8_t* sK = smem + C::OFF_K;
   uint8_t* sV = smem + C::OFF_V;
   uint8_t* sDS = smem + C::OFF_DS;
-  float* sVec = reinterpret_cast<float*>(smem + C::OFF_VEC);  // [NST][2][BM]
+  float* sVec = reinterpret_cast<float*>(smem + C::OFF_VEC);  // [C::NST][2][BM]
   Bars* bars = reinterpret_cast<Bars*>(smem + C::OFF_BAR);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -225,7 +232,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
     mbar_init(&bars->kv_empty, 1);
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < C::NST; ++s) {
       mbar_init(&bars->q_full[s], 1);
       mbar_init(&bars->q_empty[s], 1);
     }
@@ -283,9 +290,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       int g = 0;      // query tiles (Q, dO) loaded so far, over all items
       int nkv = 0;    // items whose K and V were loaded
       int dog = 0;    // dO tiles loaded
-      // loads of one query tile: Q, the LSE2 / D rows into stage g % NST, dO
+      // loads of one query tile: Q, the LSE2 / D rows into stage g % C::NST, dO
       auto load_tile = [&](const Item& w, int it) -> bool {
-        const int st = g % NST, round = g / NST;
+        const int st = g % C::NST, round = g / C::NST;
         const int i = w.i0 + it % w.nqi, bh = w.bhq0 + it / w.nqi;
         if (round > 0 && !mbar_wait(&bars->q_empty[st], (round - 1) & 1, 32)) return false;
         uint8_t* sQ = smem + C::OFF_Q + st * C::TILE;
@@ -345,9 +352,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       }
       // no copy into this CTA's shared memory may still be in flight at exit
       if (nkv > 0) mbar_wait(&bars->kv_full, (nkv - 1) & 1, 33);
-      for (int s = 0; s < NST && s < g; ++s) {
-        const int last = s + ((g - 1 - s) / NST) * NST;
-        mbar_wait(&bars->q_full[s], (last / NST) & 1, 34);
+      for (int s = 0; s < C::NST && s < g; ++s) {
+        const int last = s + ((g - 1 - s) / C::NST) * C::NST;
+        mbar_wait(&bars->q_full[s], (last / C::NST) & 1, 34);
       }
       if (dog > 0) mbar_wait(&bars->do_full, (dog - 1) & 1, 48);
     }
@@ -359,7 +366,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // per-tile one, and an MN-major operand differs only in LBO.
     const uint64_t d0 = sdesc_sw128(smem_u32(smem), 16, 1024);
     constexpr uint64_t kToMn = (uint64_t)((C::CHUNK >> 4) - 1) << 16;  // LBO 16 B -> CHUNK
-    auto q_desc = [&](int gt) { return sdesc_at(opaque(d0), C::OFF_Q + (gt % NST) * C::TILE); };
+    auto q_desc = [&](int gt) { return sdesc_at(opaque(d0), C::OFF_Q + (gt % C::NST) * C::TILE); };
     // S^T = K Q^T  (keys x queries), K = d
     auto issue_s = [&](int gt) {
       const uint64_t dq = q_desc(gt), dk = opaque(d0);
@@ -406,11 +413,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const Item w = decode_item(p, item);
       if (lane == 0) {
         ok = mbar_wait(&bars->kv_full, r & 1, 35);
-        if (ok) ok = mbar_wait(&bars->q_full[g % NST], (g / NST) & 1, 36);
+        if (ok) ok = mbar_wait(&bars->q_full[g % C::NST], (g / C::NST) & 1, 36);
         if (ok) {
           tc_fence_after();
           issue_s(g);
-          if (kDQ && g > 0) ok = mbar_wait(&bars->dq_empty, (g - 1) & 1, 37);
+          if (kDQ && C::DQ_SHARED && g > 0) ok = mbar_wait(&bars->dq_empty, (g - 1) & 1, 37);
         }
         if (ok) ok = mbar_wait(&bars->do_full, g & 1, 49);
         if (ok) {
@@ -418,7 +425,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           issue_dp();
         }
         for (int it = 0; it < w.niter && ok; ++it, ++g) {
-          const int st = g % NST;
+          const int st = g % C::NST;
           const bool more = it + 1 < w.niter;
           ok = mbar_wait(&bars->p_full, g & 1, 46);
           if (!ok) break;
@@ -426,7 +433,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           issue_dv(it == 0);
           if (!kDQ && !more) mma_commit(&bars->kv_empty);  // the item's last reads of K and V are issued
           if (more) {
-            ok = mbar_wait(&bars->q_full[(g + 1) % NST], ((g + 1) / NST) & 1, 36);
+            ok = mbar_wait(&bars->q_full[(g + 1) % C::NST], ((g + 1) / C::NST) & 1, 36);
             if (!ok) break;
             tc_fence_after();
             issue_s(g + 1);
@@ -445,11 +452,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           }
           mma_commit(&bars->q_empty[st]);
           if constexpr (kDQ) {
-            // dQ_part = dS K  (queries x d), K = 128 keys; written over dP^T
+            // dQ_part = dS K  (queries x d), K = 128 keys; written over dP^T at
+            // d = 128.  In its own columns (d = 64) it overwrites the previous
+            // tile's partial dQ, once the reduce warps have drained that.
+            if (!C::DQ_SHARED && g > 0) {
+              ok = mbar_wait(&bars->dq_empty, (g - 1) & 1, 37);
+              if (!ok) break;
+              tc_fence_after();
+            }
             const uint64_t dmn = opaque(d0) + kToMn;
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk)
-              mma_ss(tmem + C::T_DP, sdesc_at(dmn, C::OFF_DS + kk * 2048), sdesc_at(dmn, C::OFF_K + kk * 2048),
+              mma_ss(tmem + C::T_DQ, sdesc_at(dmn, C::OFF_DS + kk * 2048), sdesc_at(dmn, C::OFF_K + kk * 2048),
                      C::IDESC_DQ, kk > 0);
             mma_commit(&bars->dq_full);
             if (!more) mma_commit(&bars->kv_empty);
@@ -459,7 +473,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
           if (more) {
             // dP^T(i+1) overwrites the columns dQ(i) was drained from; without dQ
             // the compute warps have read dP^T(i) before they published dS(i)
-            if constexpr (kDQ) ok = mbar_wait(&bars->dq_empty, g & 1, 37);
+            if constexpr (kDQ && C::DQ_SHARED) ok = mbar_wait(&bars->dq_empty, g & 1, 37);
             if (ok) ok = mbar_wait(&bars->do_full, (g + 1) & 1, 49);
             if (!ok) break;
             tc_fence_after();
@@ -499,10 +513,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const int kr = w.j * BN + r;
       const bool key_ok = kr < p.Nk;
       for (int it = 0; it < w.niter && ok; ++it, ++g) {
-        const int i = w.i0 + it % w.nqi, st = g % NST;
+        const int i = w.i0 + it % w.nqi, st = g % C::NST;
         const uint32_t lse2 = smem_u32(sVec + st * 2 * BM) + h * 64 * 4;  // -LSE*log2(e), my columns
         const uint32_t dsv = lse2 + BM * 4;                                // -D, my columns
-        ok = mbar_wait(&bars->q_full[st], (g / NST) & 1, 40);
+        ok = mbar_wait(&bars->q_full[st], (g / C::NST) & 1, 40);
         if (ok) ok = mbar_wait(&bars->s_full, g & 1, 41);
         if (!ok) break;
         tc_fence_after();
@@ -656,7 +670,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     // in turn) and lane 0 adds the buffer into the fp32 accumulator with one
     // bulk tensor reduce-add.  No per-thread global atomics.
     const int qw = warp % 4;
-    const uint32_t tQ = tmem + ((uint32_t)(qw * 32) << 16) + C::T_DP;
+    const uint32_t tQ = tmem + ((uint32_t)(qw * 32) << 16) + C::T_DQ;
     const uint32_t stg0 = smem_u32(smem + C::OFF_STG + qw * 2 * C::STG_BYTES);
     bool ok = true;
     int chunk = 0, g = 0;
