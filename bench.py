@@ -480,35 +480,72 @@ def run_ours(args, w, world, rank, local):
     else:
         t_extras_end = t_timed_end
 
-    # end to end through the public Python API: pinned host inputs in, results out
+    # End to end through the public Python API: every step copies its inputs in
+    # from pinned host memory, runs the forward (and backward) and copies every
+    # result back to pinned host memory.  Steps are pipelined as an input
+    # pipeline would run them: two sets of device buffers, uploads on one
+    # stream, the kernels on another and downloads on a third, so step s+1's
+    # uploads overlap step s's downloads (PCIe carries both directions at once).
     hq, hk, hv = (t.pin_memory() for t in prob.host[:3])
     hdo = prob.host[3].pin_memory() if w.backward else None
-    outs = [prob.o, prob.lse] + ([prob.dq, prob.dk, prob.dv] if w.backward else [])
-    houts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv) + ((hdo,) if w.backward else ()))
-    d2h = sum(t.numel() * t.element_size() for t in houts)
+    hins = [hq, hk, hv] + ([hdo] if w.backward else [])
 
-    def e2e_step():
-        prob.q.copy_(hq, non_blocking=True)
-        prob.k.copy_(hk, non_blocking=True)
-        prob.v.copy_(hv, non_blocking=True)
-        fa.forward(prob.q, prob.k, prob.v, causal=w.causal, scale=w.scale, out=prob.o, lse=prob.lse)
+    def dev_set():
+        ins = [torch.empty_like(prob.q), torch.empty_like(prob.k), torch.empty_like(prob.v)]
         if w.backward:
-            prob.do.copy_(hdo, non_blocking=True)
-            fa.backward(prob.q, prob.k, prob.v, prob.o, prob.do, prob.lse, causal=w.causal, scale=w.scale,
-                        dq=prob.dq, dk=prob.dk, dv=prob.dv, workspace=prob.ws)
-        for h, d_ in zip(houts, outs):
-            h.copy_(d_, non_blocking=True)
+            ins.append(torch.empty_like(prob.do))
+        outs_ = [torch.empty_like(prob.o), torch.empty_like(prob.lse)]
+        if w.backward:
+            outs_ += [torch.empty_like(prob.dq), torch.empty_like(prob.dk), torch.empty_like(prob.dv)]
+        return ins, outs_
 
-    for _ in range(max(1, args.warmup)):
-        e2e_step()
+    sets = [dev_set(), dev_set()]
+    houts = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in sets[0][1]]
+    h2d = sum(t.numel() * t.element_size() for t in hins)
+    d2h = sum(t.numel() * t.element_size() for t in houts)
+    s_up, s_run, s_down = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in_ready", "in_free", "out_ready", "out_free")}
+    used = [False, False]
+
+    def e2e_step(s_idx):
+        b = s_idx % 2
+        ins, outs_ = sets[b]
+        with torch.cuda.stream(s_up):
+            if used[b]:
+                s_up.wait_event(ev["in_free"][b])  # the kernels of step s-2 are done with these inputs
+            for dst, src in zip(ins, hins):
+                dst.copy_(src, non_blocking=True)
+            ev["in_ready"][b].record(s_up)
+        with torch.cuda.stream(s_run):
+            s_run.wait_event(ev["in_ready"][b])
+            if used[b]:
+                s_run.wait_event(ev["out_free"][b])  # step s-2's results have been copied out
+            q_, k_, v_ = ins[:3]
+            fa.forward(q_, k_, v_, causal=w.causal, scale=w.scale, out=outs_[0], lse=outs_[1])
+            if w.backward:
+                fa.backward(q_, k_, v_, outs_[0], ins[3], outs_[1], causal=w.causal, scale=w.scale,
+                            dq=outs_[2], dk=outs_[3], dv=outs_[4], workspace=prob.ws)
+            ev["in_free"][b].record(s_run)
+            ev["out_ready"][b].record(s_run)
+        with torch.cuda.stream(s_down):
+            s_down.wait_event(ev["out_ready"][b])
+            for h, d_ in zip(houts, outs_):
+                h.copy_(d_, non_blocking=True)
+            ev["out_free"][b].record(s_down)
+        used[b] = True
+
+    for i in range(max(1, args.warmup)):
+        e2e_step(i)
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(n):
-        e2e_step()
-    e1.record()
+    # the timed region: from before the first upload to after the last download
+    e0.record(s_up)
+    s_run.wait_event(e0)
+    s_down.wait_event(e0)
+    for i in range(n):
+        e2e_step(i)
+    e1.record(s_down)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n, world)
     barrier(world)
