@@ -547,6 +547,19 @@ def run_ours(args, w, world, rank, local):
         e2e_step(i)
     e1.record(s_down)
     torch.cuda.synchronize()
+    # every step had the same inputs: the last step's downloaded results must be
+    # those of the kernel-only runs (dQ, summed by reduce-adds in a varying
+    # order, to fp32 rounding), or the pipeline's ordering is wrong
+    ref_outs = [prob.o, prob.lse] + ([prob.dq, prob.dk, prob.dv] if w.backward else [])
+    for name, h, d_ in zip(("O", "LSE", "dQ", "dK", "dV"), houts, ref_outs):
+        ref_h = d_.cpu()
+        if name == "dQ":
+            rel = float((h.float() - ref_h.float()).norm() / ref_h.float().norm().clamp_min(1e-30))
+            ok_e2e = rel < 1e-3
+        else:
+            ok_e2e = torch.equal(h, ref_h)
+        if not ok_e2e:
+            raise RuntimeError(f"end-to-end {name} differs from the kernel-only result")
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n, world)
     barrier(world)
     fa.check_device_status()
