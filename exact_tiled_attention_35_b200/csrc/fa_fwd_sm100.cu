@@ -61,7 +61,7 @@ constexpr int kItemReaders = 9;    // MMA issuer and the 8 softmax warps
 constexpr int kSchedSlots = 256;   // ticket counters, one per launch in flight
 constexpr unsigned int kHeldTag = 0xFFFFFFFFu;  // owner tag of no launch (diagnostics)
 // Register split (setmaxnreg).  The launch gives every thread 168 registers,
-// 384 * 168 = 64512 in all; the shares sum to 128 * (2*208 + 88) = 64512.
+// 384 * 168 = 64512 in all; the shares sum to 128 * (2*216 + 72) = 64512.
 // 216 per softmax thread leaves its code without spills (208 spilled 20 bytes);
 // the producer and the MMA issuer fit in 72.
 constexpr int kRegsSoftmax = 216;  // warpgroups 0 and 1
