@@ -370,33 +370,6 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
   return (uint32_t)r;
 }
 
-// exp2 of two values on the FMA pipe instead of the MUFU unit, for part of the
-// exponentials (the two units then share the work).  Cody-Waite range
-// reduction: n = round(x) and f = x - n in [-1/2, 1/2] (one add of 1.5 * 2^23
-// leaves n in the low mantissa bits; subtracting it again gives n exactly), then
-// 2^f by a degree-3 polynomial whose coefficients are the float32 rounding of
-// the minimax (Remez) fit of relative error on [-1/2, 1/2] (csrc/exp2_poly_fit.py;
-// maximum relative error 7.5e-5), and finally n is added to the exponent field.
-// x is clamped at -120 first, so -inf and large negative inputs give about
-// 2^-120 rather than 0: callers use it only where no element is masked.
-__device__ __forceinline__ void ex2_poly_x2(float x0, float x1, float& y0, float& y1) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0x1.fff692p-1f, c1 = 0x1.62f31ap-1f, c2 = 0x1.f0de1ap-3f, c3 = 0x1.c3f76p-5f;
-  const uint64_t x = f2_pack(fmaxf(x0, -120.f), fmaxf(x1, -120.f));
-  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));
-  const uint64_t n = f2_add(t, f2_pack(-kRound, -kRound));
-  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);
-  uint64_t q = f2_fma(f2_pack(c3, c3), f, f2_pack(c2, c2));
-  q = f2_fma(q, f, f2_pack(c1, c1));
-  q = f2_fma(q, f, f2_pack(c0, c0));
-  float t0, t1, q0, q1;
-  f2_unpack(t, t0, t1);
-  f2_unpack(q, q0, q1);
-  // q * 2^n: the low bits of t hold n; shifted to the exponent field they add n
-  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
-  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));

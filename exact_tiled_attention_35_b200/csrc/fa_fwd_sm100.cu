@@ -42,7 +42,6 @@
 
 #include <algorithm>
 #include <atomic>
-#include <type_traits>
 
 #include "fa_device.cuh"
 #include "fa_kernels.h"
@@ -70,10 +69,6 @@ static_assert(128 * (2 * kRegsSoftmax + kRegsControl) <= NTHREADS * 168,
               "register split exceeds the launch allocation");
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-
-// Exponentials of unmasked tiles computed on the FMA pipe (ex2_poly_x2) rather
-// than the MUFU unit: this many of every 8 pairs of a row's keys.
-constexpr int kEmuPairsPer8 = 0;
 
 // Tile geometry for head dimension D and element type (F8: e4m3, else bf16).
 // A 128-row tile is stored as NCHUNK column chunks of SW bytes per row, each in
@@ -546,21 +541,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
       const uint64_t c2 = f2_pack(c, c), nmc2 = f2_pack(-mc, -mc);
       uint64_t sum2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
       // Exponentials of one half (64 keys), packed for the P V MMA (bf16 pairs, or
-      // e4m3 quadruples); in a tile without masked keys some pairs are computed on
-      // the FMA pipe, spread evenly over the row.
-      auto exps = [&](auto emu, int half, uint32_t(&pk)[32]) {
-        constexpr bool kEmu = decltype(emu)::value;
+      // e4m3 quadruples).
+      auto exps = [&](int half, uint32_t(&pk)[32]) {
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const int e = half * 64 + 2 * i;
-          float x0, x1, p0, p1;
+          float x0, x1;
           f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), c2, nmc2), x0, x1);
-          if (kEmu && ((i * kEmuPairsPer8) % 8) < kEmuPairsPer8) {
-            ex2_poly_x2(x0, x1, p0, p1);
-          } else {
-            p0 = ex2(x0);
-            p1 = ex2(x1);
-          }
+          const float p0 = ex2(x0), p1 = ex2(x1);
           sum2[i % 2] = f2_add(sum2[i % 2], f2_pack(p0, p1));
           if constexpr (F8) {
             const uint32_t h = pack_e4m3x2(p0, p1);
@@ -575,10 +563,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
-        if (need_mask)
-          exps(std::false_type{}, half, pk);
-        else
-          exps(std::true_type{}, half, pk);
+        exps(half, pk);
         if constexpr (F8) {
           uint32_t pk16[16];
 #pragma unroll
